@@ -1,0 +1,163 @@
+/*
+ * fldce.h -- C ABI of the fused linear diffusion cross-entropy for B200 (sm_100a).
+ *
+ * What it computes (the page "fused_linear_diffusion_cross_entropy.py":
+ * fused_linear_cross_entropy_forward, cross_entropy_kernel steps 1-6 and
+ * fused_linear_cross_entropy_backward).  For hidden states H[N,D], LM-head
+ * weight W[V,D], targets y[N], masking probabilities p[N], logit scale s,
+ * label smoothing eps, normaliser T and upstream gradient g:
+ *
+ *   z[n,v]  = s * <H[n], W[v]>                (never written to memory)
+ *   lse[n]  = log sum_v exp z[n,v]
+ *   CE[n]   = (1-eps)(lse[n] - z[n,y_n]) + eps (lse[n] - mean_v z[n,v])
+ *   loss[n] = CE[n] / (p_n T),  loss = sum_n loss[n]     (0 for ignored n)
+ *   G[n,v]  = g s (softmax[n,v] - eps/V - (1-eps)[v=y_n]) / (p_n T)
+ *   dH = G W,  dW = G^T H
+ *
+ * A token is ignored when y_n == ignore_index; a target outside [0,V) that
+ * is not ignore_index is a caller error: it is counted (err_count) and the
+ * token is treated as ignored.  p_mask of an ignored token is never read.
+ *
+ * Conventions for every entry point:
+ *   - Return value: FLDCE_OK (0) or a negative FLDCE_ERR_* code; nothing is
+ *     launched when an argument check fails.  fldce_strerror() names a code.
+ *   - Pointers named "device" must be device memory of the current CUDA
+ *     device; the caller allocates and owns every buffer.  The library never
+ *     allocates device memory and never synchronises the host: all work is
+ *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Layouts are dense row-major.  bf16 is IEEE bfloat16 (stored as
+ *     uint16), fp32 is IEEE binary32.  Device pointers of H, W, dH, dW, G
+ *     and the workspace must be 16-byte aligned; D must be a multiple of 8.
+ *   - The handle holds host state only (the configuration); it is not
+ *     thread-safe: use one handle per host thread, or serialise calls.
+ */
+#ifndef FLDCE_H_
+#define FLDCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define FLDCE_OK                    0
+#define FLDCE_ERR_INVALID_ARG      -1  /* null/ill-sized argument, N > max_N, ... */
+#define FLDCE_ERR_UNSUPPORTED      -2  /* D % 8 != 0, unknown dtype or flag      */
+#define FLDCE_ERR_WORKSPACE        -3  /* workspace too small or misaligned       */
+#define FLDCE_ERR_CUDA             -4  /* a CUDA runtime call or launch failed    */
+#define FLDCE_ERR_DEVICE           -5  /* current device is not compute 10.x      */
+#define FLDCE_ERR_ALIGN            -6  /* a device pointer is not 16-byte aligned */
+
+/* Element types of H, W, dH and (unless FLDCE_FLAG_DW_FP32) dW. */
+#define FLDCE_BF16  0   /* tcgen05 tensor-core path, fp32 accumulation        */
+#define FLDCE_FP32  1   /* CUDA-core fp32 path (small problems, 1e-5 parity)  */
+
+/* Configuration flags. */
+#define FLDCE_FLAG_DW_FP32  0x1u  /* dW is written as fp32 instead of the dtype */
+
+typedef struct fldce_plan* fldce_handle;
+
+typedef struct {
+    int32_t dtype;            /* FLDCE_BF16 or FLDCE_FP32                         */
+    uint32_t flags;           /* FLDCE_FLAG_*                                     */
+    int64_t D;                /* hidden size, > 0, multiple of 8                  */
+    int64_t V;                /* vocabulary size, > 0                             */
+    int64_t max_N;            /* largest token count passed to a call, > 0        */
+    int64_t chunk_N;          /* tokens per internal chunk; 0 = library's choice  */
+    float logit_scale;        /* s (the page's logit_scale), finite and nonzero   */
+    float label_smoothing;    /* eps in [0, 1]                                    */
+    int64_t ignore_index;     /* the page's ignore_index, usually -100            */
+} fldce_config;
+
+/*
+ * fldce_create -- validate `cfg` and build a plan (host memory only).
+ *   out             [out] the new handle; unchanged on error.
+ *   cfg             [in]  configuration; copied, the caller keeps ownership.
+ *   workspace_bytes [out, may be NULL] device workspace needed by a call
+ *                   with N = cfg->max_N (calls with smaller N need no more).
+ * Errors: INVALID_ARG (null out/cfg, a size <= 0, eps outside [0,1],
+ * logit_scale zero or not finite, chunk_N < 0), UNSUPPORTED (dtype, flags,
+ * D % 8 != 0).
+ */
+int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_bytes);
+
+/*
+ * fldce_workspace_size -- device workspace bytes a call with N tokens needs.
+ * Errors: INVALID_ARG (null handle/bytes, N < 0 or N > max_N).
+ */
+int fldce_workspace_size(fldce_handle h, int64_t N, size_t* bytes);
+
+/*
+ * fldce_fwd_bwd -- loss and both gradients in one asynchronous call
+ * (the page's FusedLinearCrossEntropyFunction.forward computes the loss and
+ * all gradients at once; its backward only multiplies them by grad_out,
+ * which here is folded in).
+ *
+ *   H        [device, in]  [N, D] dtype.
+ *   W        [device, in]  [V, D] dtype.
+ *   target   [device, in]  [N] int64.
+ *   p_mask   [device, in]  [N] fp32, or NULL for p = 1 (ordinary CE).
+ *   N        tokens, 0 <= N <= max_N.  N == 0 writes loss = 0 and dW = 0.
+ *   total    T > 0 is used as given ('mean' over an explicit normaliser;
+ *            'sum' is T = 1); T <= 0 means the count of non-ignored,
+ *            in-range targets, computed on the device (no host sync).
+ *   grad_out g, the upstream gradient of the scalar loss (1 for a loss that
+ *            ends the graph).
+ *   loss            [device, out] 1 fp32: sum_n loss[n] (fixed-order sum).
+ *   loss_per_token  [device, out, may be NULL] [N] fp32 loss[n].
+ *   lse             [device, out, may be NULL] [N] fp32 lse[n] (every row).
+ *   argmax          [device, out, may be NULL] [N] int32 lowest v with
+ *                   z[n,v] = max_v z[n,v] (every row).
+ *   dH       [device, out] [N, D] dtype; overwritten.
+ *   dW       [device, out] [V, D] dtype (fp32 with FLDCE_FLAG_DW_FP32);
+ *            overwritten (not accumulated into).
+ *   workspace        [device] scratch of at least fldce_workspace_size(N)
+ *                    bytes, 256-byte aligned; contents need no initialisation
+ *                    and are undefined afterwards.  Calls that share a
+ *                    workspace must be ordered on the GPU (same stream).
+ *   workspace_bytes  its size.
+ *   err_count [device, out, may be NULL] 2 int32: [0] = number of targets
+ *             outside [0, V) that are not ignore_index; [1] = device error
+ *             bits, 0 when every kernel completed (1 = a pipeline wait timed
+ *             out after 4 s and the results are invalid).
+ *   stream    cudaStream_t to enqueue on.
+ * Errors: INVALID_ARG, ALIGN, WORKSPACE, DEVICE, CUDA (launch failure).
+ */
+int fldce_fwd_bwd(fldce_handle h,
+                  const void* H, const void* W, const int64_t* target,
+                  const float* p_mask, int64_t N, float total, float grad_out,
+                  float* loss, float* loss_per_token, float* lse, int32_t* argmax,
+                  void* dH, void* dW,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* err_count, void* stream);
+
+/*
+ * fldce_forward -- the loss sweep alone, for evaluation: loss, and
+ * optionally loss_per_token / lse / argmax, with no gradients (the page's
+ * logsumexp_fwd plus cross_entropy_kernel step 4, without steps 5-6).
+ * Arguments mean what they mean for fldce_fwd_bwd.  Needs no more
+ * workspace than fldce_fwd_bwd.
+ */
+int fldce_forward(fldce_handle h,
+                  const void* H, const void* W, const int64_t* target,
+                  const float* p_mask, int64_t N, float total,
+                  float* loss, float* loss_per_token, float* lse, int32_t* argmax,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* err_count, void* stream);
+
+/* fldce_destroy -- free the plan's host memory.  NULL is accepted. */
+int fldce_destroy(fldce_handle h);
+
+/* fldce_strerror -- static English text for a status code. */
+const char* fldce_strerror(int status);
+
+/* fldce_version -- library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fldce_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLDCE_H_ */

@@ -1,0 +1,441 @@
+// fldce_api.cu -- host side of the C ABI declared in include/fldce.h.
+//
+// One call runs, on the caller's stream and without any host synchronisation:
+//   k_count_targets                      all N tokens (the normaliser T)
+//   per token chunk [r0, r0 + rows):
+//     sweep 1  GEMM H W^T + LseEpi       per (row, vocab tile) partial lse
+//     k_merge_rows                       lse, loss[n], gradient coefficient
+//     sweep 2  GEMM H W^T + GEpi         G (bf16) for the chunk
+//     dH GEMM  G W                       dH rows of the chunk
+//     dW GEMM  G^T H                     dW (accumulated over chunks)
+//   k_finish                             fixed-order loss sum, error count
+// The chunk loop is the page's fused_linear_cross_entropy_forward loop over
+// token chunks; it bounds the workspace.  bf16 runs on tcgen05 tensor cores;
+// fp32 runs the CUDA-core GEMM of kernels.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "../../include/fldce.h"
+#include "kernels.cuh"
+
+using namespace fldce;
+
+namespace {
+
+constexpr int kVersion = 100;          // 0.1.0
+constexpr int kBN = 256;               // vocab tile of the tensor-core sweeps
+constexpr int kStages = 4;
+constexpr size_t kAlign = 256;
+constexpr size_t kGBudget = size_t(1) << 32;   // G buffer per chunk: at most 4 GiB
+
+using CfgKK = GemmCfg<kBN, kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
+using CfgKM = GemmCfg<kBN, kStages, false, true>;    // dH: G (K-major), W (MN-major)
+using CfgMM = GemmCfg<kBN, kStages, true, true>;     // dW: G^T (MN-major), H (MN-major)
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct DeviceInfo {
+    int major = -1;
+    int sms = 0;
+};
+
+bool device_info(DeviceInfo* out) {
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < 64 && cache[dev].major >= 0) { *out = cache[dev]; return true; }
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return false;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return false;
+    if (dev < 64) cache[dev] = d;
+    *out = d;
+    return true;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] matrix with row stride
+// `ld` elements; box = [box_outer, box_inner], 128-byte swizzle, zero fill
+// outside the extent.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+              uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class Cfg, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64_t N, int64_t K,
+                        int n_fastest, const typename Epi::Params& ep, int32_t* err, int sms,
+                        cudaStream_t st) {
+    GemmGeom g;
+    g.tiles_m = (int)cdiv(M, Cfg::BM);
+    g.tiles_n = (int)cdiv(N, Cfg::BN);
+    g.k_iters = (int)cdiv(K, Cfg::BK);
+    g.num_tiles = g.tiles_m * g.tiles_n;
+    g.n_fastest = n_fastest;
+    if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
+    auto kern = umma_gemm_kernel<Cfg, Epi>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int grid = std::min(g.num_tiles, sms);
+    kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(a, b, g, ep, err);
+    return cudaGetLastError();
+}
+
+template <class Epi>
+cudaError_t launch_simt(const float* A, int64_t sam, int64_t sak, const float* B, int64_t sbn,
+                        int64_t sbk, int M, int64_t N, int K, const Epi& epi, cudaStream_t st) {
+    if (M <= 0 || N <= 0) return cudaSuccess;
+    dim3 grid((unsigned)cdiv(N, kSimtTile), (unsigned)cdiv(M, kSimtTile));
+    simt_gemm_kernel<Epi><<<grid, 256, 0, st>>>(A, sam, sak, B, sbn, sbk, M, N, K, epi);
+    return cudaGetLastError();
+}
+
+struct Layout {
+    size_t cnt, part_ml, part_sz, part_am, zy, row_lse2, row_gcoef, row_y, loss_tok, G, dw_acc;
+    size_t total;
+    int64_t C;        // rows per chunk buffer
+    int64_t nchunks;
+};
+
+}  // namespace
+
+struct fldce_plan {
+    fldce_config cfg;
+    int64_t chunk;    // tokens per chunk
+    int64_t Vpad;     // row stride of G (elements)
+    int tile_v;       // vocab tile width of the partial statistics
+    int64_t n_vt;     // number of vocab tiles
+    size_t elt;       // bytes per element of H / W / G
+};
+
+namespace {
+
+bool dw_out_fp32(const fldce_plan* p) {
+    return p->cfg.dtype == FLDCE_FP32 || (p->cfg.flags & FLDCE_FLAG_DW_FP32) != 0;
+}
+
+Layout make_layout(const fldce_plan* p, int64_t N) {
+    Layout L{};
+    const int64_t C = std::max<int64_t>(1, std::min<int64_t>(p->chunk, N));
+    L.C = C;
+    L.nchunks = N > 0 ? cdiv(N, p->chunk) : 0;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = round_up(off + bytes, kAlign);
+        return o;
+    };
+    const size_t nv = (size_t)p->n_vt * (size_t)C;
+    L.cnt = take(sizeof(Counters));
+    L.part_ml = take(nv * 8);
+    L.part_sz = take(nv * 4);
+    L.part_am = take(nv * 4);
+    L.zy = take(C * 4);
+    L.row_lse2 = take(C * 4);
+    L.row_gcoef = take(C * 4);
+    L.row_y = take(C * 4);
+    L.loss_tok = take(std::max<int64_t>(N, 1) * 4);
+    L.G = take((size_t)C * p->Vpad * p->elt);
+    const bool acc = L.nchunks > 1 && !dw_out_fp32(p);
+    L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
+    L.total = off;
+    return L;
+}
+
+bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+
+int check_device(DeviceInfo* d) {
+    if (!device_info(d)) return FLDCE_ERR_CUDA;
+    if (d->major != 10) return FLDCE_ERR_DEVICE;
+    return FLDCE_OK;
+}
+
+// The shared body of fldce_fwd_bwd and fldce_forward.
+int run(fldce_handle h, const void* H, const void* W, const int64_t* target, const float* p_mask,
+        int64_t N, float total, float grad_out, float* loss, float* loss_tok_out, float* lse_out,
+        int32_t* argmax_out, void* dH, void* dW, void* workspace, size_t workspace_bytes,
+        int32_t* err_count, void* stream, bool backward) {
+    if (h == nullptr || loss == nullptr || N < 0 || N > h->cfg.max_N) return FLDCE_ERR_INVALID_ARG;
+    if (N > 0 && (H == nullptr || W == nullptr || target == nullptr)) return FLDCE_ERR_INVALID_ARG;
+    if (backward && (dW == nullptr || (N > 0 && dH == nullptr))) return FLDCE_ERR_INVALID_ARG;
+    if (!std::isfinite(total) || !std::isfinite(grad_out)) return FLDCE_ERR_INVALID_ARG;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+        return FLDCE_ERR_WORKSPACE;
+    if (!aligned16(H) || !aligned16(W) || (backward && (!aligned16(dH) || !aligned16(dW))))
+        return FLDCE_ERR_ALIGN;
+    const Layout L = make_layout(h, N);
+    if (workspace_bytes < L.total) return FLDCE_ERR_WORKSPACE;
+    DeviceInfo dev;
+    if (int s = check_device(&dev)) return s;
+
+    const fldce_config& cfg = h->cfg;
+    const int64_t D = cfg.D, V = cfg.V;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    Counters* cnt = reinterpret_cast<Counters*>(ws + L.cnt);
+    float2* part_ml = reinterpret_cast<float2*>(ws + L.part_ml);
+    float* part_sz = reinterpret_cast<float*>(ws + L.part_sz);
+    int32_t* part_am = reinterpret_cast<int32_t*>(ws + L.part_am);
+    float* zy = reinterpret_cast<float*>(ws + L.zy);
+    float* row_lse2 = reinterpret_cast<float*>(ws + L.row_lse2);
+    float* row_gcoef = reinterpret_cast<float*>(ws + L.row_gcoef);
+    int32_t* row_y = reinterpret_cast<int32_t*>(ws + L.row_y);
+    float* loss_tok = loss_tok_out != nullptr ? loss_tok_out
+                                              : reinterpret_cast<float*>(ws + L.loss_tok);
+    const bool bf16 = cfg.dtype == FLDCE_BF16;
+    const float s = cfg.logit_scale, eps = cfg.label_smoothing;
+    const float c = s * 1.4426950408889634f;
+
+#define FLDCE_CUDA(x)                                  \
+    do {                                               \
+        if ((x) != cudaSuccess) return FLDCE_ERR_CUDA; \
+    } while (0)
+
+    FLDCE_CUDA(cudaMemsetAsync(cnt, 0, sizeof(Counters), st));
+    if (N > 0) {
+        const int blocks = (int)std::min<int64_t>(cdiv(N, 256), 4 * (int64_t)dev.sms);
+        k_count_targets<<<blocks, 256, 0, st>>>(target, N, V, cfg.ignore_index, cnt);
+        FLDCE_CUDA(cudaGetLastError());
+    } else if (backward) {
+        FLDCE_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * D * (dw_out_fp32(h) ? 4 : h->elt), st));
+    }
+
+    const bool fp32_dw = dw_out_fp32(h);
+    float* dw_ws = fp32_dw ? static_cast<float*>(dW) : reinterpret_cast<float*>(ws + L.dw_acc);
+
+    CUtensorMap mW_k, mW_mn;
+    if (bf16 && N > 0) {
+        if (!make_map(&mW_k, W, D, V, D, 64, kBN)) return FLDCE_ERR_CUDA;
+        if (backward && !make_map(&mW_mn, W, D, V, D, 64, 64)) return FLDCE_ERR_CUDA;
+    }
+
+    for (int64_t ci = 0; ci < L.nchunks; ++ci) {
+        const int64_t r0 = ci * h->chunk;
+        const int rows = (int)std::min<int64_t>(h->chunk, N - r0);
+        const int64_t* tgt = target + r0;
+
+        LseEpi::Params lp;
+        lp.c = c;
+        lp.s = s;
+        lp.V = V;
+        lp.rows = rows;
+        lp.ld_part = (int)L.C;
+        lp.target = tgt;
+        lp.part_ml = part_ml;
+        lp.part_sz = eps > 0.f ? part_sz : nullptr;
+        lp.part_am = argmax_out != nullptr ? part_am : nullptr;
+        lp.zy = zy;
+
+        CUtensorMap mH_k, mH_mn, mG_k, mG_mn;
+        if (bf16) {
+            const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
+            if (!make_map(&mH_k, Hc, D, rows, D, 64, 128)) return FLDCE_ERR_CUDA;
+            FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, lp, &cnt->dev_err,
+                                                   dev.sms, st)));
+        } else {
+            const float* Hc = static_cast<const float*>(H) + r0 * D;
+            SimtLse e{lp};
+            FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
+                                   e, st));
+        }
+
+        MergeParams mp;
+        mp.rows = rows;
+        mp.ld_part = (int)L.C;
+        mp.n_vt = (int)h->n_vt;
+        mp.V = V;
+        mp.ignore_index = cfg.ignore_index;
+        mp.s = s;
+        mp.eps = eps;
+        mp.total = total;
+        mp.grad_out = grad_out;
+        mp.target = tgt;
+        mp.p_mask = p_mask != nullptr ? p_mask + r0 : nullptr;
+        mp.part_ml = part_ml;
+        mp.part_sz = eps > 0.f ? part_sz : nullptr;
+        mp.part_am = argmax_out != nullptr ? part_am : nullptr;
+        mp.zy = zy;
+        mp.cnt = cnt;
+        mp.loss_tok = loss_tok + r0;
+        mp.lse_out = lse_out != nullptr ? lse_out + r0 : nullptr;
+        mp.am_out = argmax_out != nullptr ? argmax_out + r0 : nullptr;
+        mp.row_lse2 = backward ? row_lse2 : nullptr;
+        mp.row_gcoef = row_gcoef;
+        mp.row_y = row_y;
+        k_merge_rows<<<(unsigned)cdiv(rows, 128), 128, 0, st>>>(mp);
+        FLDCE_CUDA(cudaGetLastError());
+        if (!backward) continue;
+
+        const int mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : (ci + 1 < L.nchunks || fp32_dw ? 2 : 3));
+        if (bf16) {
+            __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(ws + L.G);
+            GEpi::Params gp;
+            gp.c = c;
+            gp.V = V;
+            gp.ldg = h->Vpad;
+            gp.rows = rows;
+            gp.lse2 = row_lse2;
+            gp.gcoef = row_gcoef;
+            gp.ycol = row_y;
+            gp.eps_over_V = eps / (float)V;
+            gp.one_minus_eps = 1.f - eps;
+            gp.G = G;
+            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, gp, &cnt->dev_err,
+                                                 dev.sms, st)));
+            if (!make_map(&mG_k, G, V, rows, h->Vpad, 64, 128)) return FLDCE_ERR_CUDA;
+            if (!make_map(&mG_mn, G, V, rows, h->Vpad, 64, 64)) return FLDCE_ERR_CUDA;
+            const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
+            if (!make_map(&mH_mn, Hc, D, rows, D, 64, 64)) return FLDCE_ERR_CUDA;
+
+            StoreEpi::Params hp;
+            hp.rows = rows;
+            hp.cols = D;
+            hp.ldo = D;
+            hp.out = static_cast<__nv_bfloat16*>(dH) + r0 * D;
+            hp.ws = nullptr;
+            hp.mode = 0;
+            hp.out_fp32 = 0;
+            FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1, hp,
+                                                     &cnt->dev_err, dev.sms, st)));
+            StoreEpi::Params wp;
+            wp.rows = (int)V;
+            wp.cols = D;
+            wp.ldo = D;
+            wp.out = dW;
+            wp.ws = dw_ws;
+            wp.mode = mode;
+            wp.out_fp32 = fp32_dw ? 1 : 0;
+            FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, wp,
+                                                     &cnt->dev_err, dev.sms, st)));
+        } else {
+            float* G = reinterpret_cast<float*>(ws + L.G);
+            const float* Hc = static_cast<const float*>(H) + r0 * D;
+            SimtG ge{c, V, h->Vpad, rows, row_lse2, row_gcoef, row_y, eps / (float)V, 1.f - eps, G};
+            FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
+                                   ge, st));
+            SimtStore hs{rows, D, D, static_cast<float*>(dH) + r0 * D, nullptr, 0};
+            FLDCE_CUDA(launch_simt(G, h->Vpad, 1, static_cast<const float*>(W), 1, D, rows, D,
+                                   (int)V, hs, st));
+            SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, mode == 3 ? 2 : mode};
+            FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
+        }
+    }
+
+    k_finish<<<1, 1024, 0, st>>>(loss_tok, N, cnt, loss, err_count);
+    FLDCE_CUDA(cudaGetLastError());
+#undef FLDCE_CUDA
+    return FLDCE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_bytes) {
+    if (out == nullptr || cfg == nullptr) return FLDCE_ERR_INVALID_ARG;
+    if (cfg->D <= 0 || cfg->V <= 0 || cfg->max_N <= 0 || cfg->chunk_N < 0)
+        return FLDCE_ERR_INVALID_ARG;
+    if (!(cfg->label_smoothing >= 0.f && cfg->label_smoothing <= 1.f))
+        return FLDCE_ERR_INVALID_ARG;
+    if (!std::isfinite(cfg->logit_scale) || cfg->logit_scale == 0.f) return FLDCE_ERR_INVALID_ARG;
+    if (cfg->dtype != FLDCE_BF16 && cfg->dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
+    if ((cfg->flags & ~FLDCE_FLAG_DW_FP32) != 0) return FLDCE_ERR_UNSUPPORTED;
+    if (cfg->D % 8 != 0) return FLDCE_ERR_UNSUPPORTED;
+    if (cfg->V > (int64_t(1) << 31) - 1 || cfg->max_N > (int64_t(1) << 31) - 1 ||
+        cfg->D > (int64_t(1) << 31) - 1)
+        return FLDCE_ERR_UNSUPPORTED;
+    fldce_plan* p = new (std::nothrow) fldce_plan;
+    if (p == nullptr) return FLDCE_ERR_INVALID_ARG;
+    p->cfg = *cfg;
+    p->elt = cfg->dtype == FLDCE_BF16 ? 2 : 4;
+    p->Vpad = (int64_t)round_up((size_t)cfg->V, 8);
+    p->tile_v = cfg->dtype == FLDCE_BF16 ? kBN : kSimtTile;
+    p->n_vt = cdiv(cfg->V, p->tile_v);
+    int64_t chunk = cfg->chunk_N;
+    if (chunk == 0) {
+        chunk = (int64_t)(kGBudget / ((size_t)p->Vpad * p->elt)) / 128 * 128;
+        chunk = std::max<int64_t>(chunk, 128);
+    }
+    p->chunk = std::min<int64_t>(chunk, cfg->max_N);
+    if (workspace_bytes != nullptr) *workspace_bytes = make_layout(p, cfg->max_N).total;
+    *out = p;
+    return FLDCE_OK;
+}
+
+int fldce_workspace_size(fldce_handle h, int64_t N, size_t* bytes) {
+    if (h == nullptr || bytes == nullptr || N < 0 || N > h->cfg.max_N) return FLDCE_ERR_INVALID_ARG;
+    *bytes = make_layout(h, N).total;
+    return FLDCE_OK;
+}
+
+int fldce_fwd_bwd(fldce_handle h, const void* H, const void* W, const int64_t* target,
+                  const float* p_mask, int64_t N, float total, float grad_out, float* loss,
+                  float* loss_per_token, float* lse, int32_t* argmax, void* dH, void* dW,
+                  void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream) {
+    return run(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse, argmax, dH,
+               dW, workspace, workspace_bytes, err_count, stream, true);
+}
+
+int fldce_forward(fldce_handle h, const void* H, const void* W, const int64_t* target,
+                  const float* p_mask, int64_t N, float total, float* loss, float* loss_per_token,
+                  float* lse, int32_t* argmax, void* workspace, size_t workspace_bytes,
+                  int32_t* err_count, void* stream) {
+    return run(h, H, W, target, p_mask, N, total, 1.f, loss, loss_per_token, lse, argmax, nullptr,
+               nullptr, workspace, workspace_bytes, err_count, stream, false);
+}
+
+int fldce_destroy(fldce_handle h) {
+    delete h;
+    return FLDCE_OK;
+}
+
+const char* fldce_strerror(int status) {
+    switch (status) {
+        case FLDCE_OK: return "ok";
+        case FLDCE_ERR_INVALID_ARG: return "invalid argument";
+        case FLDCE_ERR_UNSUPPORTED: return "unsupported configuration (dtype, flags or D % 8 != 0)";
+        case FLDCE_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
+        case FLDCE_ERR_CUDA: return "CUDA runtime error or failed launch";
+        case FLDCE_ERR_DEVICE: return "current device is not a compute capability 10.x GPU";
+        case FLDCE_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int fldce_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,515 @@
+// kernels.cuh -- epilogues of the tcgen05 GEMM, the per-row kernels, and the
+// fp32 CUDA-core path of the fused linear diffusion cross-entropy.
+//
+// Notation (the page "fused_linear_diffusion_cross_entropy.py"): acc = <H[n], W[v]>
+// is the raw fp32 accumulator, z = s * acc the logit, c = s * log2(e), so that
+// t = acc * c = z * log2(e) lives in the base-2 domain where the hardware
+// exponential ex2 works.  Running statistics are kept in that domain:
+// m2 = max t, l = sum 2^(t - m2), and lse = (m2 + log2 l) * ln 2.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "umma_gemm.cuh"
+
+namespace fldce {
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ======================================================================
+// Epilogue 1 (sweep 1): per-row partial logsumexp of one vocab tile.
+// logsumexp_fwd_kernel keeps one (max, log-sum-exp) per row and vocab block;
+// here each (row, vocab tile) keeps (m2, l) plus, when asked, the sum of the
+// raw logits (label smoothing), the tile argmax, and the target logit when
+// the target falls in the tile.  Columns >= V (TMA zero fill) are excluded.
+// ======================================================================
+struct LseEpi {
+    struct Params {
+        float c;                 // s * log2(e)
+        float s;                 // logit scale
+        int64_t V;
+        int rows;                // tokens in this chunk
+        int ld_part;             // row stride of the partial arrays (chunk capacity)
+        const int64_t* target;   // chunk's targets
+        float2* part_ml;         // [n_vt][ld_part] (m2, l)
+        float* part_sz;          // [n_vt][ld_part] sum of acc, or null
+        int32_t* part_am;        // [n_vt][ld_part] argmax column, or null
+        float* zy;               // [ld_part] target logit z[n, y_n]
+    };
+
+    template <int BN>
+    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
+                                               const AccRow& acc) {
+        const int m = mt * 128 + row;
+        const int64_t n0 = (int64_t)nt * BN;
+        const bool live = m < p.rows;
+        int yrel = -1;
+        if (live) {
+            const int64_t y = p.target[m];
+            if (y >= n0 && y < n0 + BN && y < p.V) yrel = (int)(y - n0);
+        }
+        const int ncols = (int)((p.V - n0) < BN ? (p.V - n0) : BN);
+        float mx = -CUDART_INF_F, l = 0.f, sz = 0.f, zyv = 0.f, amv = -CUDART_INF_F;
+        int am = 0;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            uint32_t r[32];
+            acc.load(j, r);
+            if (j == BN / 32 - 1) acc.release();
+            float t[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) t[i] = __uint_as_float(r[i]) * p.c;
+            if (32 * j + 32 > ncols) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (32 * j + i >= ncols) t[i] = -CUDART_INF_F;
+            }
+            float cm0 = fmaxf(t[0], t[1]), cm1 = fmaxf(t[2], t[3]);
+#pragma unroll
+            for (int i = 4; i < 32; i += 4) {
+                cm0 = fmaxf(cm0, fmaxf(t[i], t[i + 1]));
+                cm1 = fmaxf(cm1, fmaxf(t[i + 2], t[i + 3]));
+            }
+            const float nm = fmaxf(mx, fmaxf(cm0, cm1));
+            if (p.part_am != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (t[i] > amv) { amv = t[i]; am = 32 * j + i; }
+            }
+            if (p.part_sz != nullptr) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    if (32 * j + i < ncols) a0 += __uint_as_float(r[i]);
+                    if (32 * j + i + 1 < ncols) a1 += __uint_as_float(r[i + 1]);
+                }
+                sz += a0 + a1;
+            }
+            if ((unsigned)(yrel - 32 * j) < 32u) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i == yrel - 32 * j) zyv = __uint_as_float(r[i]);
+            }
+            float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                e0 += ex2(t[i] - nm);
+                e1 += ex2(t[i + 1] - nm);
+                e2 += ex2(t[i + 2] - nm);
+                e3 += ex2(t[i + 3] - nm);
+            }
+            l = l * ex2(mx - nm) + ((e0 + e1) + (e2 + e3));
+            mx = nm;
+        }
+        if (live) {
+            const size_t o = (size_t)nt * p.ld_part + m;
+            p.part_ml[o] = make_float2(mx, l);
+            if (p.part_sz != nullptr) p.part_sz[o] = sz;
+            if (p.part_am != nullptr) p.part_am[o] = (int32_t)(n0 + am);
+            if (yrel >= 0) p.zy[m] = zyv * p.s;
+        }
+    }
+};
+
+// ======================================================================
+// Epilogue 2 (sweep 2): the gradient of the logits, rounded once to bf16.
+// cross_entropy_kernel steps 5-6 and the backward's grad_out:
+//   G = gcoef * (2^(t - lse2) - eps/V) - gcoef * (1 - eps) [v = y],
+//   gcoef = g s / (p T), exactly 0 for ignored tokens and columns >= V.
+// ======================================================================
+struct GEpi {
+    struct Params {
+        float c;
+        int64_t V;
+        int64_t ldg;             // row stride of G in elements (multiple of 8)
+        int rows;
+        const float* lse2;       // [chunk] lse in base-2 units
+        const float* gcoef;      // [chunk]
+        const int32_t* ycol;     // [chunk] validated target or -1
+        float eps_over_V;
+        float one_minus_eps;
+        __nv_bfloat16* G;        // [chunk][ldg]
+    };
+
+    template <int BN>
+    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
+                                               const AccRow& acc) {
+        const int m = mt * 128 + row;
+        const int64_t n0 = (int64_t)nt * BN;
+        const bool live = m < p.rows;
+        float gc = 0.f, L2 = 0.f;
+        int yrel = -1;
+        if (live) {
+            gc = p.gcoef[m];
+            if (gc != 0.f) {
+                L2 = p.lse2[m];
+                const int y = p.ycol[m];
+                if (y >= n0 && y < n0 + BN) yrel = (int)(y - n0);
+            }
+        }
+        const float base = gc * p.eps_over_V;
+        const float tcorr = gc * p.one_minus_eps;
+        const int ncols = (int)((p.V - n0) < BN ? (p.V - n0) : BN);
+        const int scols = (int)((p.ldg - n0) < BN ? (p.ldg - n0) : BN);
+        __nv_bfloat16* grow = p.G + (size_t)(live ? m : 0) * p.ldg + n0;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            uint32_t r[32];
+            acc.load(j, r);
+            if (j == BN / 32 - 1) acc.release();
+            float g[32];
+            if (gc != 0.f) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    g[i] = fmaf(gc, ex2(fmaf(__uint_as_float(r[i]), p.c, -L2)), -base);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) g[i] = 0.f;
+            }
+            if ((unsigned)(yrel - 32 * j) < 32u) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i == yrel - 32 * j) g[i] -= tcorr;
+            }
+            if (32 * j + 32 > ncols) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (32 * j + i >= ncols) g[i] = 0.f;
+            }
+            if (live) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (32 * j + 8 * q < scols) {
+                        uint4 v;
+                        v.x = pack_bf16x2(g[8 * q + 0], g[8 * q + 1]);
+                        v.y = pack_bf16x2(g[8 * q + 2], g[8 * q + 3]);
+                        v.z = pack_bf16x2(g[8 * q + 4], g[8 * q + 5]);
+                        v.w = pack_bf16x2(g[8 * q + 6], g[8 * q + 7]);
+                        *reinterpret_cast<uint4*>(grow + 32 * j + 8 * q) = v;
+                    }
+                }
+            }
+        }
+    }
+};
+
+// ======================================================================
+// Epilogue 3: dH / dW tiles.  mode 0: out = acc; 1: ws = acc; 2: ws += acc;
+// 3: out = ws + acc (fp32 workspace ws carries dW across token chunks).
+// ======================================================================
+struct StoreEpi {
+    struct Params {
+        int rows;                // valid output rows
+        int64_t cols;            // valid output columns
+        int64_t ldo;             // row stride of out / ws (elements)
+        void* out;               // bf16 or fp32
+        float* ws;               // fp32 accumulator (modes 1-3)
+        int mode;
+        int out_fp32;
+    };
+
+    template <int BN>
+    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
+                                               const AccRow& acc) {
+        const int m = mt * 128 + row;
+        const int64_t n0 = (int64_t)nt * BN;
+        const bool live = m < p.rows;
+        const size_t rbase = (size_t)(live ? m : 0) * p.ldo + n0;
+#pragma unroll 1
+        for (int j = 0; j < BN / 32; ++j) {
+            uint32_t r[32];
+            acc.load(j, r);
+            if (j == BN / 32 - 1) acc.release();
+            if (!live) continue;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t col = n0 + 32 * j + 8 * q;
+                if (col >= p.cols) continue;
+                const size_t o = rbase + 32 * j + 8 * q;
+                float* x = v + 8 * q;
+                if (p.mode >= 2) {
+                    const float4 a = *reinterpret_cast<const float4*>(p.ws + o);
+                    const float4 b = *reinterpret_cast<const float4*>(p.ws + o + 4);
+                    x[0] += a.x; x[1] += a.y; x[2] += a.z; x[3] += a.w;
+                    x[4] += b.x; x[5] += b.y; x[6] += b.z; x[7] += b.w;
+                }
+                if (p.mode == 1 || p.mode == 2) {
+                    *reinterpret_cast<float4*>(p.ws + o) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(p.ws + o + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                } else if (p.out_fp32) {
+                    float* out = reinterpret_cast<float*>(p.out) + o;
+                    *reinterpret_cast<float4*>(out) = make_float4(x[0], x[1], x[2], x[3]);
+                    *reinterpret_cast<float4*>(out + 4) = make_float4(x[4], x[5], x[6], x[7]);
+                } else {
+                    uint4 w;
+                    w.x = pack_bf16x2(x[0], x[1]);
+                    w.y = pack_bf16x2(x[2], x[3]);
+                    w.z = pack_bf16x2(x[4], x[5]);
+                    w.w = pack_bf16x2(x[6], x[7]);
+                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) = w;
+                }
+            }
+        }
+    }
+};
+
+// ======================================================================
+// Row kernels shared by both element types.
+// ======================================================================
+struct Counters {
+    int32_t n_valid;   // targets != ignore_index and inside [0, V)
+    int32_t n_err;     // targets != ignore_index outside [0, V)
+    int32_t dev_err;   // FLDCE_DEV_ERR_* bits raised by kernels
+    int32_t pad;
+};
+
+// Count the tokens that carry a loss (the page's target.ne(ignore_index).sum(),
+// without the host round trip) and the malformed targets.
+__global__ void k_count_targets(const int64_t* __restrict__ target, int64_t N, int64_t V,
+                                int64_t ignore_index, Counters* cnt) {
+    int valid = 0, bad = 0;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t y = target[i];
+        if (y != ignore_index) {
+            if (y >= 0 && y < V) ++valid; else ++bad;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        valid += __shfl_xor_sync(0xffffffffu, valid, o);
+        bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        if (valid) atomicAdd(&cnt->n_valid, valid);
+        if (bad) atomicAdd(&cnt->n_err, bad);
+    }
+}
+
+struct MergeParams {
+    int rows;                 // tokens in this chunk
+    int ld_part;              // partial row stride
+    int n_vt;                 // vocab tiles
+    int64_t V;
+    int64_t ignore_index;
+    float s, eps, total, grad_out;
+    const int64_t* target;    // chunk's targets
+    const float* p_mask;      // chunk's p_mask or null
+    const float2* part_ml;
+    const float* part_sz;     // null when eps == 0
+    const int32_t* part_am;   // null when argmax is not wanted
+    const float* zy;
+    const Counters* cnt;
+    float* loss_tok;          // chunk's per-token loss
+    float* lse_out;           // chunk's lse output or null
+    int32_t* am_out;          // chunk's argmax output or null
+    float* row_lse2;          // [chunk] for sweep 2 (null in forward-only mode)
+    float* row_gcoef;
+    int32_t* row_y;
+};
+
+// Split-V merge: lse = M + log sum_k l_k 2^(m_k - M) (logsumexp_fwd's second
+// logsumexp; the tensor-parallel tutorial's sum of per-shard denominators),
+// then the per-token loss (cross_entropy_kernel step 4 and the
+// label-smoothing block) and the per-token gradient coefficient.
+__global__ void k_merge_rows(MergeParams p) {
+    const int m = blockIdx.x * blockDim.x + threadIdx.x;
+    if (m >= p.rows) return;
+    float M2 = -CUDART_INF_F;
+    int kbest = 0;
+    for (int k = 0; k < p.n_vt; ++k) {
+        const float v = p.part_ml[(size_t)k * p.ld_part + m].x;
+        if (v > M2) { M2 = v; kbest = k; }
+    }
+    float L = 0.f;
+    for (int k = 0; k < p.n_vt; ++k) {
+        const float2 ml = p.part_ml[(size_t)k * p.ld_part + m];
+        L += ml.y * exp2f(ml.x - M2);
+    }
+    const float lse2 = M2 + log2f(L);
+    const float lse = lse2 * 0.69314718055994530942f;
+    const int64_t y = p.target[m];
+    const bool valid = (y != p.ignore_index) && y >= 0 && y < p.V;
+    float loss = 0.f, gcoef = 0.f;
+    if (valid) {
+        const float T = p.total > 0.f ? p.total : (float)p.cnt->n_valid;
+        const float pm = p.p_mask != nullptr ? p.p_mask[m] : 1.f;
+        const float coef = 1.f / (pm * T);
+        float ce = lse - p.zy[m];
+        if (p.eps > 0.f) {
+            float sz = 0.f;
+            for (int k = 0; k < p.n_vt; ++k) sz += p.part_sz[(size_t)k * p.ld_part + m];
+            const float meanz = p.s * sz / (float)p.V;
+            ce = (1.f - p.eps) * ce + p.eps * (lse - meanz);
+        }
+        loss = ce * coef;
+        gcoef = p.grad_out * p.s * coef;
+    }
+    p.loss_tok[m] = loss;
+    if (p.lse_out != nullptr) p.lse_out[m] = lse;
+    if (p.am_out != nullptr) p.am_out[m] = p.part_am[(size_t)kbest * p.ld_part + m];
+    if (p.row_lse2 != nullptr) {
+        p.row_lse2[m] = lse2;
+        p.row_gcoef[m] = gcoef;
+        p.row_y[m] = valid ? (int32_t)y : -1;
+    }
+}
+
+// loss = sum_n loss[n] in a fixed order (one block, fp64 partials), so the
+// scalar is bit-reproducible run to run; also publishes the malformed-target
+// count and the device error bits (a timed-out wait) in err_count[0..1].
+__global__ void k_finish(const float* __restrict__ loss_tok, int64_t N, const Counters* cnt,
+                         float* loss, int32_t* err_count) {
+    __shared__ double red[1024];
+    double acc = 0.0;
+    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)loss_tok[i];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+        if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        *loss = (float)red[0];
+        if (err_count != nullptr) {
+            err_count[0] = cnt->n_err;
+            err_count[1] = cnt->dev_err;
+        }
+    }
+}
+
+// ======================================================================
+// fp32 CUDA-core path: a 64x64-tile SIMT GEMM whose tile is staged in shared
+// memory and handed to an epilogue.  Used for the fp32 element type, where
+// the tensor cores' tf32 would not meet fp32 accuracy.
+// ======================================================================
+constexpr int kSimtTile = 64;
+
+struct SimtLse {
+    LseEpi::Params p;
+    __device__ void operator()(float (*C)[kSimtTile + 1], int m0, int64_t n0, int nt) const {
+        const int r = threadIdx.x;
+        if (r >= kSimtTile) return;
+        const int m = m0 + r;
+        if (m >= p.rows) return;
+        const int ncols = (int)((p.V - n0) < kSimtTile ? (p.V - n0) : kSimtTile);
+        float mx = -CUDART_INF_F, sz = 0.f;
+        int am = 0;
+        for (int i = 0; i < ncols; ++i) {
+            const float t = C[r][i] * p.c;
+            if (t > mx) { mx = t; am = i; }
+            sz += C[r][i];
+        }
+        float l = 0.f;
+        for (int i = 0; i < ncols; ++i) l += exp2f(C[r][i] * p.c - mx);
+        const size_t o = (size_t)nt * p.ld_part + m;
+        p.part_ml[o] = make_float2(mx, l);
+        if (p.part_sz != nullptr) p.part_sz[o] = sz;
+        if (p.part_am != nullptr) p.part_am[o] = (int32_t)(n0 + am);
+        const int64_t y = p.target[m];
+        if (y >= n0 && y < n0 + ncols) p.zy[m] = C[r][y - n0] * p.s;
+    }
+};
+
+struct SimtG {
+    float c;
+    int64_t V, ldg;
+    int rows;
+    const float* lse2;
+    const float* gcoef;
+    const int32_t* ycol;
+    float eps_over_V, one_minus_eps;
+    float* G;
+    __device__ void operator()(float (*C)[kSimtTile + 1], int m0, int64_t n0, int) const {
+        for (int idx = threadIdx.x; idx < kSimtTile * kSimtTile; idx += blockDim.x) {
+            const int r = idx / kSimtTile, i = idx % kSimtTile;
+            const int m = m0 + r;
+            const int64_t v = n0 + i;
+            if (m >= rows || v >= ldg) continue;
+            const float gc = gcoef[m];
+            float g = 0.f;
+            if (gc != 0.f && v < V) {
+                g = gc * exp2f(C[r][i] * c - lse2[m]) - gc * eps_over_V;
+                if (v == ycol[m]) g -= gc * one_minus_eps;
+            }
+            G[(size_t)m * ldg + v] = g;
+        }
+    }
+};
+
+struct SimtStore {
+    int rows;
+    int64_t cols, ldo;
+    float* out;
+    float* ws;
+    int mode;
+    __device__ void operator()(float (*C)[kSimtTile + 1], int m0, int64_t n0, int) const {
+        for (int idx = threadIdx.x; idx < kSimtTile * kSimtTile; idx += blockDim.x) {
+            const int r = idx / kSimtTile, i = idx % kSimtTile;
+            const int m = m0 + r;
+            const int64_t col = n0 + i;
+            if (m >= rows || col >= cols) continue;
+            const size_t o = (size_t)m * ldo + col;
+            float x = C[r][i];
+            if (mode >= 2) x += ws[o];
+            if (mode == 1 || mode == 2) ws[o] = x; else out[o] = x;
+        }
+    }
+};
+
+// C[m, n] = sum_k A[m*sam + k*sak] * B[n*sbn + k*sbk]
+template <class Epi>
+__global__ void __launch_bounds__(256)
+simt_gemm_kernel(const float* __restrict__ A, int64_t sam, int64_t sak,
+                 const float* __restrict__ B, int64_t sbn, int64_t sbk, int M, int64_t N, int K,
+                 Epi epi) {
+    __shared__ float As[16][kSimtTile + 4];
+    __shared__ float Bs[16][kSimtTile + 4];
+    __shared__ float Cs[kSimtTile][kSimtTile + 1];
+    const int m0 = blockIdx.y * kSimtTile;
+    const int64_t n0 = (int64_t)blockIdx.x * kSimtTile;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        for (int e = threadIdx.x; e < 16 * kSimtTile; e += 256) {
+            const int mm = e % kSimtTile, kk = e / kSimtTile;
+            const int gm = m0 + mm, gk = k0 + kk;
+            As[kk][mm] = (gm < M && gk < K) ? A[(int64_t)gm * sam + (int64_t)gk * sak] : 0.f;
+            const int64_t gn = n0 + mm;
+            Bs[kk][mm] = (gn < N && gk < K) ? B[gn * sbn + (int64_t)gk * sbk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) Cs[ty * 4 + i][tx * 4 + j] = acc[i][j];
+    __syncthreads();
+    epi(Cs, m0, n0, (int)blockIdx.x);
+}
+
+}  // namespace fldce

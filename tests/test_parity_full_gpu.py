@@ -1,0 +1,81 @@
+"""GPU parity at the full workload sizes, in the launch configuration bench.py
+times (default chunking, argmax on).  The oracle computes what it can one
+row at a time: every sampled token's lse, loss and dH row, every sampled
+vocabulary row of dW where the whole batch's lse is affordable (mid and
+headline), and properties that hold at any size everywhere:
+
+* ignored tokens: loss and dH row exactly zero (every token, not a sample);
+* loss == sum of loss_per_token;
+* every row of G sums to zero, so the column sums of dW vanish
+  (|sum_v dW[v, :]| small against sum_v |dW[v, :]|).
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.fldce_oracle as O
+from linear_diffusion_cross_b200 import synth
+from tests._parity import (GRAD_TOL, LOSS_RTOL, check_rows, f64, maxabs_err, oracle_inputs,
+                           oracle_kw, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+N_SAMPLE_ROWS = 192
+N_SAMPLE_VOCAB = 128
+
+
+def _global_checks(wl, g):
+    ign = (wl.target == wl.ignore_index).numpy()
+    lt = g["loss_per_token"].double().numpy()
+    assert np.all(lt[ign] == 0.0)
+    dH = g["dH"]
+    assert torch.count_nonzero(dH[torch.from_numpy(ign)]) == 0
+    loss = float(g["loss"][0])
+    assert abs(loss - lt.sum()) <= 1e-5 * abs(lt.sum())
+    assert int(g["err"][0]) == 0 and int(g["err"][1]) == 0
+    dW = g["dW"].float()
+    colsum = dW.double().sum(0).abs()
+    colabs = dW.double().abs().sum(0)
+    ratio = float((colsum / colabs.clamp_min(1e-30)).max())
+    assert ratio < 2e-2, f"dW column sums not ~0: {ratio}"
+    return ratio
+
+
+def _rows(wl, seed):
+    must = [0, wl.N - 1]
+    return synth.sample_rows(wl.N, N_SAMPLE_ROWS, seed, must).numpy()
+
+
+@pytest.mark.parametrize("name", ["mid", "headline", "ragged", "large"])
+def test_full_size(name):
+    t0 = time.time()
+    wl = synth.make(name, 0)
+    g = run_gpu(wl)
+    H, W, y, p = oracle_inputs(wl)
+    valid, _ = O.valid_tokens(y, wl.V, wl.ignore_index)
+    T = O.resolve_total(wl.total, valid)
+    info = {"gen_and_gpu_s": time.time() - t0}
+    info["dW_colsum_ratio"] = _global_checks(wl, g)
+
+    rows = _rows(wl, 1)
+    t1 = time.time()
+    ref = O.fldce_rows(H, W, y, p, rows, total=T, **oracle_kw(wl))
+    info.update(check_rows(wl, g, ref, rows, "bf16"))
+    info["oracle_rows_s"] = time.time() - t1
+
+    if name in ("mid", "headline"):
+        must = [wl.V - 1] + [int(v) for v in y[valid][:8]]
+        vr = synth.sample_rows(wl.V, N_SAMPLE_VOCAB, 2, must).numpy()
+        t2 = time.time()
+        dWr, lse_all, lt_all = O.fldce_dw_rows(H, W, y, p, vr, total=T, **oracle_kw(wl))
+        info["oracle_dw_s"] = time.time() - t2
+        e_dw = maxabs_err(f64(g["dW"])[vr], dWr)
+        assert e_dw <= GRAD_TOL["bf16"], f"dW err {e_dw}"
+        info["dW"] = e_dw
+        loss_ref = float(lt_all.sum())
+        loss = float(g["loss"][0])
+        assert abs(loss - loss_ref) <= LOSS_RTOL * abs(loss_ref), (loss, loss_ref)
+        info["loss"] = abs(loss - loss_ref) / abs(loss_ref)
+    print(name, info)
