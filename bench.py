@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the fused linear diffusion cross-entropy (loss + dH + dW) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fldce|reference]
+                    [--workload headline|mid|ragged|large|tiny]
+
+One step = one fldce_fwd_bwd call over one batch of the workload: sweep 1
+(logits + online logsumexp), the split-V merge, sweep 2 (logits recomputed,
+G formed), dH = G W and dW = G^T H.  The default workload is the headline
+one: N = 8192 tokens (2 x 4096), D = 2560, V = 151936, bf16, block-diffusion
+masking (blocks of 4 tokens share t ~ U(1e-3, 1)), total = N, seed 0.
+
+Rank 0 prints one JSON line.  `value` is whole-job tokens/s with inputs
+resident in HBM (W = 778 MB is larger than the 126 MB L2, so no flush is
+needed between steps); `e2e` is the same metric with the inputs copied from
+pinned host memory and the loss copied back inside every step; `roofline`
+is the dominant kernel's algorithmic TFLOP/s (2 N D V per GEMM launch) over
+its CUDA-event duration inside the timed region; `cpu_baseline` times the
+float64 oracle on a bounded token sample on the host cores.
+
+Under torchrun (N > 1) each rank runs its own batch (weak scaling) with the
+weight replicated; after every step dW and the loss are summed across ranks
+with NCCL (the data-parallel exchange step).  `--impl reference` times the
+float64 oracle (the reference arm of this comparison) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_diffusion_cross_b200 import binding as B  # noqa: E402
+from linear_diffusion_cross_b200 import synth  # noqa: E402
+
+METRIC = "fwd+bwd tokens/s and TFLOP/s at N=8192,D=2560,V=151936 bf16; % of bf16 TC peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_KINDS = ("lse_sweep", "g_sweep", "dh_gemm", "dw_gemm")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(name: str, r: synth.Recipe) -> str:
+    t = f"per block of {r.t_block} tokens" if r.t_block else "per sequence"
+    total = "count of non-ignored tokens" if r.total_is_count else "N"
+    extra = f", {int(r.peaky_frac * 100)}% of W rows x{int(r.peaky_mult)}" if r.peaky_frac else ""
+    dt = "bf16" if r.dtype == torch.bfloat16 else "fp32"
+    return (f"{name}: N={r.N} ({r.batch}x{r.seq}), D={r.D}, V={r.V}, {dt}; H~N(0,1), "
+            f"W~N(0,{r.sigma_w}^2){extra}; t~U({r.t_lo},1) {t}, token masked w.p. t "
+            f"(target~U[0,V), p_mask=t) else ignore_index=-100; label_smoothing="
+            f"{r.label_smoothing}, logit_scale={r.logit_scale}, total={total}; seed 0")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if not self.rows:
+            return None
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+_W64 = {}
+
+
+def cpu_baseline(wl, n_tokens: int):
+    """The float64 oracle on the first n_tokens tokens of the batch (full D, V)."""
+    import oracle.fldce_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    H = wl.H[:n_tokens].to(torch.float64).numpy()
+    if id(wl) not in _W64:
+        _W64.clear()
+        _W64[id(wl)] = wl.W.to(torch.float64).numpy()
+    W = _W64[id(wl)]
+    y = wl.target[:n_tokens].numpy()
+    p = wl.p_mask[:n_tokens].to(torch.float64).numpy()
+    valid, _ = O.valid_tokens(wl.target.numpy(), wl.V, wl.ignore_index)
+    T = O.resolve_total(wl.total, valid)
+    t0 = time.perf_counter()
+    O.fldce(H, W, y, p, total=T, logit_scale=wl.logit_scale,
+            label_smoothing=wl.label_smoothing, ignore_index=wl.ignore_index,
+            grad_out=wl.grad_out)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+            "sample": (f"first {n_tokens} of {wl.N} tokens, full D={wl.D} and V={wl.V}: loss, "
+                       f"lse, dH rows and their dW contribution in float64 numpy/OpenBLAS; "
+                       f"{dt:.2f} s"), "seconds": dt}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "fldce":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the float64 oracle timed on the host cores."""
+    if rank != 0:
+        return 0
+    r = synth.RECIPES[args.workload]
+    wl = synth.make(r, 0)
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        cb = cpu_baseline(wl, n_tok)
+    times = []
+    for _ in range(args.steps):
+        cb = cpu_baseline(wl, n_tok)
+        times.append(cb["seconds"])
+    tot = sum(times)
+    value = n_tok * len(times) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, r), "N": r.N, "D": r.D, "V": r.V,
+                   "step": f"float64 oracle on {n_tok} tokens of the batch"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cb["cores"],
+                         "kind": "oracle", "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fldce", "reference"], default="fldce")
+    ap.add_argument("--workload", choices=sorted(synth.RECIPES), default="headline")
+    ap.add_argument("--cpu-tokens", type=int, default=512,
+                    help="tokens in the float64 oracle's bounded sample")
+    ap.add_argument("--ref-tokens", type=int, default=128,
+                    help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    r = synth.RECIPES[args.workload]
+    wl = synth.make(r, 0)
+    N, D, V = wl.N, wl.D, wl.V
+    plan = B.Plan(D, V, N, dtype=wl.H.dtype, chunk_N=wl.chunk_n, logit_scale=wl.logit_scale,
+                  label_smoothing=wl.label_smoothing, ignore_index=wl.ignore_index, device=dev)
+    H, W = wl.H.to(dev), wl.W.to(dev)
+    y, p = wl.target.to(dev), wl.p_mask.to(dev)
+    total = wl.total if wl.total > 0 else 0.0
+    if world > 1:
+        # one mean over the whole job's tokens: every rank normalises by the
+        # job-wide count (all ranks hold the same batch here)
+        total = world * (wl.total if wl.total > 0 else wl.n_valid())
+    out = plan.outputs(N, want_argmax=False)
+    stream = torch.cuda.current_stream(dev)
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def step():
+        plan.fwd_bwd(H, W, y, p, total, 1.0, out=out, stream=stream)
+        if dist is not None:
+            dist.all_reduce(out["dW"])
+            dist.all_reduce(out["loss"])
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    err = out["err"].tolist()
+    if err != [0, 0]:
+        raise RuntimeError(f"device error counters {err}")
+
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    B.fldce_profile_begin(plan.handle, args.steps)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    prof = B.fldce_profile_end(plan.handle)
+    ms_total = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t)
+    ms = ms_total / args.steps
+    tok_s = world * N * args.steps / (ms_total / 1e3)
+    flops = 6.0 * N * D * V
+    peaks, peaks_src = load_peaks()
+
+    # dominant kernel and its roofline
+    kinds = {k: v for k, v in prof.items() if v[1] > 0}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    dom_ms = kinds[dom][0] / kinds[dom][1]
+    total_kernel_ms = sum(v[0] for v in kinds.values())
+    launches = sum(v[1] for v in kinds.values())
+    peak_key = "bf16_tflops_sustained"
+    roof = None
+    if dom in GEMM_KINDS:
+        chunks = -(-N // B.fldce_chunk_size(plan.handle))
+        fl_launch = 2.0 * N * D * V / chunks
+        ach = fl_launch / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": ach,
+                "peak": peaks[peak_key], "unit": "TFLOP/s", "frac": ach / peaks[peak_key],
+                "peak_source": f"{peaks_src} {peak_key}",
+                "frac_of_burst": ach / peaks["bf16_tflops"],
+                "flops_per_launch": fl_launch, "ms_per_launch": dom_ms,
+                "traffic": traffic_for(dom, args.workload)}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(plan, wl, total, args, dev, stream, dist)
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(wl, min(args.cpu_tokens, N))
+        cb.pop("seconds", None)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; shapes and masking of the workload)",
+            "config": {"workload": workload_desc(args.workload, r), "N": N, "D": D, "V": V,
+                       "chunk_N": B.fldce_chunk_size(plan.handle),
+                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (W is 778 MB, L2 126 MB); no flush"},
+            "tflops": world * flops / (ms / 1e3) / 1e12,
+            "tflops_executed_8NDV": world * flops * 4 / 3 / (ms / 1e3) / 1e12,
+            "pct_of_bf16_peak": 100.0 * flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "peak_bf16_tflops": peaks["bf16_tflops"], "peaks_source": peaks_src,
+            "roofline": roof,
+            "kernels_ms_per_step": {k: v[0] / args.steps for k, v in kinds.items()},
+            "kernel_share": {k: v[0] / total_kernel_ms for k, v in kinds.items()},
+            "gpu_launches": launches,
+            "e2e": e2e, "cpu_baseline": cb, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if current."""
+    path = os.path.join(ROOT, "profiles", f"ncu_{kernel}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    src = vals.get("source_sha256")
+    if src is None or src != source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_diffusion_cross_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measure_e2e(plan, wl, total, args, dev, stream, dist):
+    """Same step through the public API with host buffers: pinned host inputs
+    copied to the device and the loss copied back inside every timed step."""
+    hH = wl.H.pin_memory()
+    hW = wl.W.pin_memory()
+    hy = wl.target.pin_memory()
+    hp = wl.p_mask.pin_memory()
+    hloss = torch.empty(1, dtype=torch.float32).pin_memory()
+    dH_ = torch.empty_like(hH, device=dev)
+    dW_ = torch.empty_like(hW, device=dev)
+    dy = torch.empty_like(hy, device=dev)
+    dp = torch.empty_like(hp, device=dev)
+    out = plan.outputs(wl.N, want_argmax=False)
+    h2d = sum(t.numel() * t.element_size() for t in (hH, hW, hy, hp))
+    d2h = hloss.numel() * hloss.element_size()
+
+    def step():
+        dH_.copy_(hH, non_blocking=True)
+        dW_.copy_(hW, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        dp.copy_(hp, non_blocking=True)
+        plan.fwd_bwd(dH_, dW_, dy, dp, total, 1.0, out=out, stream=stream)
+        if dist is not None:
+            dist.all_reduce(out["dW"])
+            dist.all_reduce(out["loss"])
+        hloss.copy_(out["loss"], non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    k = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(k):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t)
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": world * wl.N * k / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k,
+            "ms_per_step": ms / k}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

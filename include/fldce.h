@@ -90,6 +90,14 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
 int fldce_workspace_size(fldce_handle h, int64_t N, size_t* bytes);
 
 /*
+ * fldce_chunk_size -- tokens per internal chunk the plan uses (the explicit
+ * chunk_N, or the library's choice: the largest multiple of 128 tokens whose
+ * G buffer stays within 4 GiB, capped at max_N).
+ * Errors: INVALID_ARG (null handle or out).
+ */
+int fldce_chunk_size(fldce_handle h, int64_t* chunk_N);
+
+/*
  * fldce_fwd_bwd -- loss and both gradients in one asynchronous call
  * (the page's FusedLinearCrossEntropyFunction.forward computes the loss and
  * all gradients at once; its backward only multiplies them by grad_out,
@@ -147,7 +155,26 @@ int fldce_forward(fldce_handle h,
                   void* workspace, size_t workspace_bytes,
                   int32_t* err_count, void* stream);
 
-/* fldce_destroy -- free the plan's host memory.  NULL is accepted. */
+/*
+ * Optional profiling window: per-kernel device time over a window of calls.
+ * fldce_profile_begin(h, max_calls) creates CUDA events (no device memory)
+ * for the next `max_calls` calls on this handle; each of those calls records
+ * an event on its stream after every kernel it launches.  Calls past the
+ * window are not recorded.  fldce_profile_end() waits for the recorded events,
+ * then fills, per kernel kind k < FLDCE_PROF_KINDS, the summed device time
+ * in ms[k] and the number of launches in launches[k] (either may be NULL),
+ * and closes the window.  The time of a kernel is the interval between the
+ * event before it and the event after it on the same stream.
+ * Errors: INVALID_ARG (null handle, max_calls <= 0), CUDA.
+ */
+#define FLDCE_PROF_KINDS 7
+int fldce_profile_begin(fldce_handle h, int max_calls);
+int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches);
+/* Name of kernel kind k ("lse_sweep", "g_sweep", "dh_gemm", ...), or NULL. */
+const char* fldce_profile_kind_name(int kind);
+
+/* fldce_destroy -- free the plan's host memory (and profiling events).
+ * NULL is accepted. */
 int fldce_destroy(fldce_handle h);
 
 /* fldce_strerror -- static English text for a status code. */

@@ -30,8 +30,10 @@ FLDCE_FP32 = 1
 FLDCE_FLAG_DW_FP32 = 0x1
 
 # every symbol include/fldce.h declares
-EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_fwd_bwd", "fldce_forward",
+EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd", "fldce_forward",
+           "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
            "fldce_destroy", "fldce_strerror", "fldce_version")
+FLDCE_PROF_KINDS = 7
 
 
 class FldceError(RuntimeError):
@@ -74,12 +76,21 @@ def load() -> ctypes.CDLL:
     lib.fldce_create.restype = ctypes.c_int
     lib.fldce_workspace_size.argtypes = [_P, _I64, ctypes.POINTER(ctypes.c_size_t)]
     lib.fldce_workspace_size.restype = ctypes.c_int
+    lib.fldce_chunk_size.argtypes = [_P, ctypes.POINTER(_I64)]
+    lib.fldce_chunk_size.restype = ctypes.c_int
     lib.fldce_fwd_bwd.argtypes = [_P, _P, _P, _P, _P, _I64, _F, _F, _P, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P, _P]
     lib.fldce_fwd_bwd.restype = ctypes.c_int
     lib.fldce_forward.argtypes = [_P, _P, _P, _P, _P, _I64, _F, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P, _P]
     lib.fldce_forward.restype = ctypes.c_int
+    lib.fldce_profile_begin.argtypes = [_P, ctypes.c_int]
+    lib.fldce_profile_begin.restype = ctypes.c_int
+    lib.fldce_profile_end.argtypes = [_P, ctypes.POINTER(ctypes.c_double),
+                                      ctypes.POINTER(ctypes.c_int32)]
+    lib.fldce_profile_end.restype = ctypes.c_int
+    lib.fldce_profile_kind_name.argtypes = [ctypes.c_int]
+    lib.fldce_profile_kind_name.restype = ctypes.c_char_p
     lib.fldce_destroy.argtypes = [_P]
     lib.fldce_destroy.restype = ctypes.c_int
     lib.fldce_strerror.argtypes = [ctypes.c_int]
@@ -139,6 +150,12 @@ def fldce_workspace_size(h: int, N: int) -> int:
     return ws.value
 
 
+def fldce_chunk_size(h) -> int:
+    c = _I64()
+    _check(load().fldce_chunk_size(h, ctypes.byref(c)), "fldce_chunk_size")
+    return c.value
+
+
 def fldce_fwd_bwd(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse,
                   argmax, dH, dW, workspace, workspace_bytes, err_count, stream=None) -> int:
     return _check(load().fldce_fwd_bwd(
@@ -153,6 +170,23 @@ def fldce_forward(h, H, W, target, p_mask, N, total, loss, loss_per_token, lse, 
         h, _ptr(H), _ptr(W), _ptr(target), _ptr(p_mask), int(N), float(total), _ptr(loss),
         _ptr(loss_per_token), _ptr(lse), _ptr(argmax), _ptr(workspace), int(workspace_bytes),
         _ptr(err_count), _stream(stream)), "fldce_forward")
+
+
+def fldce_profile_begin(h, max_calls: int) -> int:
+    return _check(load().fldce_profile_begin(h, int(max_calls)), "fldce_profile_begin")
+
+
+def fldce_profile_end(h) -> dict:
+    """{kind name: (total ms, launches)} over the window just closed."""
+    ms = (ctypes.c_double * FLDCE_PROF_KINDS)()
+    n = (ctypes.c_int32 * FLDCE_PROF_KINDS)()
+    _check(load().fldce_profile_end(h, ms, n), "fldce_profile_end")
+    return {fldce_profile_kind_name(k): (ms[k], n[k]) for k in range(FLDCE_PROF_KINDS)}
+
+
+def fldce_profile_kind_name(kind: int) -> str:
+    r = load().fldce_profile_kind_name(int(kind))
+    return r.decode() if r is not None else None
 
 
 def fldce_destroy(h) -> int:

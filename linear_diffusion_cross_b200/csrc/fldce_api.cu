@@ -20,6 +20,7 @@
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "../../include/fldce.h"
 #include "kernels.cuh"
@@ -133,6 +134,12 @@ struct Layout {
 
 }  // namespace
 
+enum ProfKind {
+    PK_COUNT = 0, PK_LSE = 1, PK_MERGE = 2, PK_G = 3, PK_DH = 4, PK_DW = 5, PK_FINISH = 6,
+    PK_GAP = -1
+};
+static_assert(FLDCE_PROF_KINDS == 7, "kinds");
+
 struct fldce_plan {
     fldce_config cfg;
     int64_t chunk;    // tokens per chunk
@@ -140,7 +147,21 @@ struct fldce_plan {
     int tile_v;       // vocab tile width of the partial statistics
     int64_t n_vt;     // number of vocab tiles
     size_t elt;       // bytes per element of H / W / G
+    // profiling window
+    std::vector<cudaEvent_t> ev;
+    std::vector<int> ev_kind;
+    size_t ev_used = 0;
+    bool prof_on = false;
 };
+
+namespace {
+// Record an event after a launch of `kind` (or a call-start gap marker).
+void prof_mark(fldce_plan* h, int kind, cudaStream_t st) {
+    if (!h->prof_on || h->ev_used >= h->ev.size()) return;
+    if (cudaEventRecord(h->ev[h->ev_used], st) != cudaSuccess) return;
+    h->ev_kind[h->ev_used++] = kind;
+}
+}  // namespace
 
 namespace {
 
@@ -226,10 +247,12 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
     } while (0)
 
     FLDCE_CUDA(cudaMemsetAsync(cnt, 0, sizeof(Counters), st));
+    prof_mark(h, PK_GAP, st);
     if (N > 0) {
         const int blocks = (int)std::min<int64_t>(cdiv(N, 256), 4 * (int64_t)dev.sms);
         k_count_targets<<<blocks, 256, 0, st>>>(target, N, V, cfg.ignore_index, cnt);
         FLDCE_CUDA(cudaGetLastError());
+        prof_mark(h, PK_COUNT, st);
     } else if (backward) {
         FLDCE_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * D * (dw_out_fp32(h) ? 4 : h->elt), st));
     }
@@ -272,6 +295,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
                                    e, st));
         }
+        prof_mark(h, PK_LSE, st);
 
         MergeParams mp;
         mp.rows = rows;
@@ -298,6 +322,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         mp.row_y = row_y;
         k_merge_rows<<<(unsigned)cdiv(rows, 128), 128, 0, st>>>(mp);
         FLDCE_CUDA(cudaGetLastError());
+        prof_mark(h, PK_MERGE, st);
         if (!backward) continue;
 
         const int mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : (ci + 1 < L.nchunks || fp32_dw ? 2 : 3));
@@ -316,6 +341,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             gp.G = G;
             FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, gp, &cnt->dev_err,
                                                  dev.sms, st)));
+            prof_mark(h, PK_G, st);
             if (!make_map(&mG_k, G, V, rows, h->Vpad, 64, 128)) return FLDCE_ERR_CUDA;
             if (!make_map(&mG_mn, G, V, rows, h->Vpad, 64, 64)) return FLDCE_ERR_CUDA;
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
@@ -331,6 +357,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             hp.out_fp32 = 0;
             FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1, hp,
                                                      &cnt->dev_err, dev.sms, st)));
+            prof_mark(h, PK_DH, st);
             StoreEpi::Params wp;
             wp.rows = (int)V;
             wp.cols = D;
@@ -341,22 +368,27 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             wp.out_fp32 = fp32_dw ? 1 : 0;
             FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, wp,
                                                      &cnt->dev_err, dev.sms, st)));
+            prof_mark(h, PK_DW, st);
         } else {
             float* G = reinterpret_cast<float*>(ws + L.G);
             const float* Hc = static_cast<const float*>(H) + r0 * D;
             SimtG ge{c, V, h->Vpad, rows, row_lse2, row_gcoef, row_y, eps / (float)V, 1.f - eps, G};
             FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
                                    ge, st));
+            prof_mark(h, PK_G, st);
             SimtStore hs{rows, D, D, static_cast<float*>(dH) + r0 * D, nullptr, 0};
             FLDCE_CUDA(launch_simt(G, h->Vpad, 1, static_cast<const float*>(W), 1, D, rows, D,
                                    (int)V, hs, st));
+            prof_mark(h, PK_DH, st);
             SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, mode == 3 ? 2 : mode};
             FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
+            prof_mark(h, PK_DW, st);
         }
     }
 
     k_finish<<<1, 1024, 0, st>>>(loss_tok, N, cnt, loss, err_count);
     FLDCE_CUDA(cudaGetLastError());
+    prof_mark(h, PK_FINISH, st);
 #undef FLDCE_CUDA
     return FLDCE_OK;
 }
@@ -402,6 +434,12 @@ int fldce_workspace_size(fldce_handle h, int64_t N, size_t* bytes) {
     return FLDCE_OK;
 }
 
+int fldce_chunk_size(fldce_handle h, int64_t* chunk_N) {
+    if (h == nullptr || chunk_N == nullptr) return FLDCE_ERR_INVALID_ARG;
+    *chunk_N = h->chunk;
+    return FLDCE_OK;
+}
+
 int fldce_fwd_bwd(fldce_handle h, const void* H, const void* W, const int64_t* target,
                   const float* p_mask, int64_t N, float total, float grad_out, float* loss,
                   float* loss_per_token, float* lse, int32_t* argmax, void* dH, void* dW,
@@ -418,7 +456,54 @@ int fldce_forward(fldce_handle h, const void* H, const void* W, const int64_t* t
                nullptr, workspace, workspace_bytes, err_count, stream, false);
 }
 
+int fldce_profile_begin(fldce_handle h, int max_calls) {
+    if (h == nullptr || max_calls <= 0) return FLDCE_ERR_INVALID_ARG;
+    const int64_t chunks = cdiv(h->cfg.max_N, h->chunk);
+    const size_t need = (size_t)max_calls * (size_t)(3 + 5 * chunks);
+    while (h->ev.size() < need) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return FLDCE_ERR_CUDA;
+        h->ev.push_back(e);
+    }
+    h->ev_kind.assign(h->ev.size(), PK_GAP);
+    h->ev_used = 0;
+    h->prof_on = true;
+    return FLDCE_OK;
+}
+
+int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches) {
+    if (h == nullptr) return FLDCE_ERR_INVALID_ARG;
+    double acc[FLDCE_PROF_KINDS] = {};
+    int32_t cnt[FLDCE_PROF_KINDS] = {};
+    h->prof_on = false;
+    if (h->ev_used > 0 && cudaEventSynchronize(h->ev[h->ev_used - 1]) != cudaSuccess)
+        return FLDCE_ERR_CUDA;
+    for (size_t i = 1; i < h->ev_used; ++i) {
+        const int k = h->ev_kind[i];
+        if (k < 0) continue;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, h->ev[i - 1], h->ev[i]) != cudaSuccess) return FLDCE_ERR_CUDA;
+        acc[k] += t;
+        cnt[k] += 1;
+    }
+    for (int k = 0; k < FLDCE_PROF_KINDS; ++k) {
+        if (ms != nullptr) ms[k] = acc[k];
+        if (launches != nullptr) launches[k] = cnt[k];
+    }
+    h->ev_used = 0;
+    return FLDCE_OK;
+}
+
+const char* fldce_profile_kind_name(int kind) {
+    static const char* names[FLDCE_PROF_KINDS] = {"count_targets", "lse_sweep", "merge",
+                                                  "g_sweep", "dh_gemm", "dw_gemm", "finish"};
+    return (kind >= 0 && kind < FLDCE_PROF_KINDS) ? names[kind] : nullptr;
+}
+
 int fldce_destroy(fldce_handle h) {
+    if (h != nullptr) {
+        for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    }
     delete h;
     return FLDCE_OK;
 }
