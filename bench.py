@@ -202,6 +202,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["fldce", "reference"], default="fldce")
     ap.add_argument("--workload", choices=sorted(synth.RECIPES), default="headline")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run the first TOKENS tokens of the workload's batch (profiling "
+                         "captures); 0 = the whole batch")
     ap.add_argument("--cpu-tokens", type=int, default=512,
                     help="tokens in the float64 oracle's bounded sample")
     ap.add_argument("--ref-tokens", type=int, default=128,
@@ -218,6 +221,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     r = synth.RECIPES[args.workload]
+    if args.tokens > 0:
+        r = synth.Recipe(**{**r.__dict__, "seq": max(1, args.tokens // r.batch)})
     wl = synth.make(r, 0)
     N, D, V = wl.N, wl.D, wl.V
     plan = B.Plan(D, V, N, dtype=wl.H.dtype, chunk_N=wl.chunk_n, logit_scale=wl.logit_scale,
