@@ -49,6 +49,7 @@ extern "C" {
 #define FLDCE_ERR_CUDA             -4  /* a CUDA runtime call or launch failed    */
 #define FLDCE_ERR_DEVICE           -5  /* current device is not compute 10.x      */
 #define FLDCE_ERR_ALIGN            -6  /* a device pointer is not 16-byte aligned */
+#define FLDCE_ERR_TOO_LARGE        -7  /* needs more scratch than the static buffer */
 
 /* Element types of H, W, dH and (unless FLDCE_FLAG_DW_FP32) dW. */
 #define FLDCE_BF16  0   /* tcgen05 tensor-core path, fp32 accumulation        */
@@ -140,6 +141,44 @@ int fldce_fwd_bwd(fldce_handle h,
                   void* dH, void* dW,
                   void* workspace, size_t workspace_bytes,
                   int32_t* err_count, void* stream);
+
+/*
+ * fldce_fwd_bwd_noalloc -- fldce_fwd_bwd for callers that cannot allocate
+ * device memory.  The paper has no counterpart to this entry point.
+ *
+ * Some callers have no way to obtain a workspace: a plugin inside a host
+ * application that owns every byte of device memory through its own pool
+ * and gives plugins no allocator, a supervisor-enforced memory budget that
+ * forbids allocations outside that pool, or a thin foreign-function binding
+ * that can only pass buffers it already has.  This entry point needs no
+ * workspace: its scratch is a static device array of
+ * FLDCE_STATIC_SCRATCH_BYTES (64 MiB) inside the library, which every GPU
+ * that loads the library holds until the process exits.  The call itself
+ * never allocates device memory.
+ *
+ * Arguments mean what they mean for fldce_fwd_bwd; the caller still
+ * provides every input and output buffer.
+ *   - Size limit: the call needs fldce_workspace_size(h, N) <=
+ *     FLDCE_STATIC_SCRATCH_BYTES, else it returns FLDCE_ERR_TOO_LARGE and
+ *     launches nothing.  A smaller chunk_N (the G buffer is chunk_N x V bf16)
+ *     and FLDCE_FLAG_DW_FP32 (no fp32 dW accumulator across chunks) make a
+ *     problem fit.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (with that device current); make that first call before any
+ *     stream capture begins.
+ *   - Sharing: every call in the process, on any handle, uses the same
+ *     array, which keeps the previous call's contents (each call clears the
+ *     counters it needs zeroed).  Calls that overlap on the GPU -- on two
+ *     streams, or from two host threads -- race on it: order them on one
+ *     stream.
+ * Errors: those of fldce_fwd_bwd, and TOO_LARGE.
+ */
+#define FLDCE_STATIC_SCRATCH_BYTES (64ull << 20)
+int fldce_fwd_bwd_noalloc(fldce_handle h,
+                          const void* H, const void* W, const int64_t* target,
+                          const float* p_mask, int64_t N, float total, float grad_out,
+                          float* loss, float* loss_per_token, float* lse, int32_t* argmax,
+                          void* dH, void* dW, int32_t* err_count, void* stream);
 
 /*
  * fldce_forward -- the loss sweep alone, for evaluation: loss, and

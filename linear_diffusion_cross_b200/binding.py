@@ -25,12 +25,15 @@ FLDCE_ERR_WORKSPACE = -3
 FLDCE_ERR_CUDA = -4
 FLDCE_ERR_DEVICE = -5
 FLDCE_ERR_ALIGN = -6
+FLDCE_ERR_TOO_LARGE = -7
+FLDCE_STATIC_SCRATCH_BYTES = 64 << 20
 FLDCE_BF16 = 0
 FLDCE_FP32 = 1
 FLDCE_FLAG_DW_FP32 = 0x1
 
 # every symbol include/fldce.h declares
-EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd", "fldce_forward",
+EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
+           "fldce_fwd_bwd_noalloc", "fldce_forward",
            "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
            "fldce_destroy", "fldce_strerror", "fldce_version")
 FLDCE_PROF_KINDS = 7
@@ -81,6 +84,9 @@ def load() -> ctypes.CDLL:
     lib.fldce_fwd_bwd.argtypes = [_P, _P, _P, _P, _P, _I64, _F, _F, _P, _P, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P, _P]
     lib.fldce_fwd_bwd.restype = ctypes.c_int
+    lib.fldce_fwd_bwd_noalloc.argtypes = [_P, _P, _P, _P, _P, _I64, _F, _F, _P, _P, _P, _P, _P,
+                                          _P, _P, _P]
+    lib.fldce_fwd_bwd_noalloc.restype = ctypes.c_int
     lib.fldce_forward.argtypes = [_P, _P, _P, _P, _P, _I64, _F, _P, _P, _P, _P, _P,
                                   ctypes.c_size_t, _P, _P]
     lib.fldce_forward.restype = ctypes.c_int
@@ -162,6 +168,16 @@ def fldce_fwd_bwd(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_to
         h, _ptr(H), _ptr(W), _ptr(target), _ptr(p_mask), int(N), float(total), float(grad_out),
         _ptr(loss), _ptr(loss_per_token), _ptr(lse), _ptr(argmax), _ptr(dH), _ptr(dW),
         _ptr(workspace), int(workspace_bytes), _ptr(err_count), _stream(stream)), "fldce_fwd_bwd")
+
+
+def fldce_fwd_bwd_noalloc(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token,
+                          lse, argmax, dH, dW, err_count, stream=None) -> int:
+    """fldce_fwd_bwd with the library's static scratch instead of a workspace,
+    for callers that cannot allocate device memory (see include/fldce.h)."""
+    return _check(load().fldce_fwd_bwd_noalloc(
+        h, _ptr(H), _ptr(W), _ptr(target), _ptr(p_mask), int(N), float(total), float(grad_out),
+        _ptr(loss), _ptr(loss_per_token), _ptr(lse), _ptr(argmax), _ptr(dH), _ptr(dW),
+        _ptr(err_count), _stream(stream)), "fldce_fwd_bwd_noalloc")
 
 
 def fldce_forward(h, H, W, target, p_mask, N, total, loss, loss_per_token, lse, argmax,

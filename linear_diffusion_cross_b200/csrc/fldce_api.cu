@@ -19,6 +19,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -448,6 +449,48 @@ int fldce_fwd_bwd(fldce_handle h, const void* H, const void* W, const int64_t* t
                dW, workspace, workspace_bytes, err_count, stream, true);
 }
 
+}  // extern "C"
+
+// Scratch of fldce_fwd_bwd_noalloc.  In host code `g_static_scratch` names a
+// host-side shadow, not device memory; the device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_static_scratch[FLDCE_STATIC_SCRATCH_BYTES];
+
+namespace {
+int static_scratch(void** out) {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return FLDCE_ERR_CUDA;
+    if (dev >= 64) return FLDCE_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+            return FLDCE_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return FLDCE_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fldce_fwd_bwd_noalloc(fldce_handle h, const void* H, const void* W, const int64_t* target,
+                          const float* p_mask, int64_t N, float total, float grad_out, float* loss,
+                          float* loss_per_token, float* lse, int32_t* argmax, void* dH, void* dW,
+                          int32_t* err_count, void* stream) {
+    if (h == nullptr || N < 0 || N > h->cfg.max_N) return FLDCE_ERR_INVALID_ARG;
+    if (make_layout(h, N).total > FLDCE_STATIC_SCRATCH_BYTES) return FLDCE_ERR_TOO_LARGE;
+    DeviceInfo dev;
+    if (int s = check_device(&dev)) return s;
+    void* scratch = nullptr;
+    if (int s = static_scratch(&scratch)) return s;
+    return run(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse, argmax, dH,
+               dW, scratch, FLDCE_STATIC_SCRATCH_BYTES, err_count, stream, true);
+}
+
 int fldce_forward(fldce_handle h, const void* H, const void* W, const int64_t* target,
                   const float* p_mask, int64_t N, float total, float* loss, float* loss_per_token,
                   float* lse, int32_t* argmax, void* workspace, size_t workspace_bytes,
@@ -517,6 +560,10 @@ const char* fldce_strerror(int status) {
         case FLDCE_ERR_CUDA: return "CUDA runtime error or failed launch";
         case FLDCE_ERR_DEVICE: return "current device is not a compute capability 10.x GPU";
         case FLDCE_ERR_ALIGN: return "device pointer not 16-byte aligned";
+        case FLDCE_ERR_TOO_LARGE:
+            return "problem needs more scratch than the 64 MiB static buffer of "
+                   "fldce_fwd_bwd_noalloc (use a smaller chunk_N, FLDCE_FLAG_DW_FP32, or "
+                   "fldce_fwd_bwd with a workspace)";
         default: return "unknown status";
     }
 }

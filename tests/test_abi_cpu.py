@@ -118,6 +118,6 @@ def test_profile_kinds(lib):
 
 
 def test_strerror(lib):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert B.fldce_strerror(code) and B.fldce_strerror(code) != "unknown status"
     assert B.fldce_strerror(-99) == "unknown status"
