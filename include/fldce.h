@@ -206,7 +206,7 @@ int fldce_forward(fldce_handle h,
  * event before it and the event after it on the same stream.
  * Errors: INVALID_ARG (null handle, max_calls <= 0), CUDA.
  */
-#define FLDCE_PROF_KINDS 7
+#define FLDCE_PROF_KINDS 8
 int fldce_profile_begin(fldce_handle h, int max_calls);
 int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches);
 /* Name of kernel kind k ("lse_sweep", "g_sweep", "dh_gemm", ...), or NULL. */

@@ -36,7 +36,7 @@ EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fw
            "fldce_fwd_bwd_noalloc", "fldce_forward",
            "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
            "fldce_destroy", "fldce_strerror", "fldce_version")
-FLDCE_PROF_KINDS = 7
+FLDCE_PROF_KINDS = 8
 
 
 class FldceError(RuntimeError):

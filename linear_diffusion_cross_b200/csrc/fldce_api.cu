@@ -32,13 +32,13 @@ namespace {
 
 constexpr int kVersion = 100;          // 0.1.0
 constexpr int kBN = 256;               // vocab tile of the tensor-core sweeps
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr size_t kAlign = 256;
 constexpr size_t kGBudget = size_t(1) << 32;   // G buffer per chunk: at most 4 GiB
 
-using CfgKK = GemmCfg<kBN, kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
-using CfgKM = GemmCfg<kBN, kStages, false, true>;    // dH: G (K-major), W (MN-major)
-using CfgMM = GemmCfg<kBN, kStages, true, true>;     // dW: G^T (MN-major), H (MN-major)
+using CfgKK = GemmCfg<kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
+using CfgKM = GemmCfg<kStages, false, true>;    // dH: G (K-major), W (MN-major)
+using CfgMM = GemmCfg<kStages, true, true>;     // dW: G^T (MN-major), H (MN-major)
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -81,30 +81,46 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a row-major [outer, inner] matrix with row stride
-// `ld` elements; box = [box_outer, box_inner], 128-byte swizzle, zero fill
-// outside the extent.
+// 2-D tensor map over a row-major [outer, inner] matrix of `elt`-byte
+// elements (bf16 or fp32) with row stride `ld` elements; box = [box_outer,
+// box_inner], 128-byte swizzle, zero fill outside the extent.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer, int elt = 2) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint64_t strides[1] = {ld * (uint64_t)elt};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUtensorMapDataType dt =
+        elt == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Store map of an output: bf16 boxes of 32 rows x 64 columns, fp32 boxes of
+// 32 rows x 32 columns (128 bytes either way).
+bool make_store_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t ld,
+                    int elt) {
+    return make_map(m, base, cols, rows, ld, elt == 4 ? 32 : 64, 32, elt);
+}
+
+// Units (tiles x K splits) per pair round; the fraction of pair slots busy.
+double wave_efficiency(int64_t units, int pairs) {
+    const int64_t rounds = (units + pairs - 1) / pairs;
+    return rounds == 0 ? 1.0 : (double)units / (double)(rounds * pairs);
 }
 
 template <class Cfg, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64_t N, int64_t K,
-                        int n_fastest, const typename Epi::Params& ep, int32_t* err, int sms,
-                        cudaStream_t st) {
+                        int n_fastest, int k_splits, const typename Epi::Params& ep, int32_t* err,
+                        int sms, cudaStream_t st) {
     GemmGeom g;
-    g.tiles_m = (int)cdiv(M, Cfg::BM);
+    g.tiles_m = (int)cdiv(M, Cfg::PAIR_M);
     g.tiles_n = (int)cdiv(N, Cfg::BN);
     g.k_iters = (int)cdiv(K, Cfg::BK);
+    g.k_splits = k_splits;
     g.num_tiles = g.tiles_m * g.tiles_n;
     g.n_fastest = n_fastest;
     if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
@@ -112,8 +128,16 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const int grid = std::min(g.num_tiles, sms);
-    kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, st>>>(a, b, g, ep, err);
+    const int pairs = std::min(g.num_tiles * g.k_splits, std::max(1, sms / 2));
+    kern<<<2 * pairs, kGemmThreads, Cfg::SMEM_BYTES, st>>>(a, b, g, ep, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, int sms, cudaStream_t st) {
+    const int64_t n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(cdiv(n8, 256), 8 * (int64_t)sms);
+    k_f32_to_bf16<<<blocks, 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), n8);
     return cudaGetLastError();
 }
 
@@ -127,7 +151,8 @@ cudaError_t launch_simt(const float* A, int64_t sam, int64_t sak, const float* B
 }
 
 struct Layout {
-    size_t cnt, part_ml, part_sz, part_am, zy, row_lse2, row_gcoef, row_y, loss_tok, G, dw_acc;
+    size_t cnt, part_ml, part_sz, part_am, zy, row_lse2, row_gcoef, row_y, loss_tok, G, dh_acc,
+        dw_acc;
     size_t total;
     int64_t C;        // rows per chunk buffer
     int64_t nchunks;
@@ -137,9 +162,9 @@ struct Layout {
 
 enum ProfKind {
     PK_COUNT = 0, PK_LSE = 1, PK_MERGE = 2, PK_G = 3, PK_DH = 4, PK_DW = 5, PK_FINISH = 6,
-    PK_GAP = -1
+    PK_CONVERT = 7, PK_GAP = -1
 };
-static_assert(FLDCE_PROF_KINDS == 7, "kinds");
+static_assert(FLDCE_PROF_KINDS == 8, "kinds");
 
 struct fldce_plan {
     fldce_config cfg;
@@ -192,6 +217,7 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
     L.row_y = take(C * 4);
     L.loss_tok = take(std::max<int64_t>(N, 1) * 4);
     L.G = take((size_t)C * p->Vpad * p->elt);
+    L.dh_acc = take(p->cfg.dtype == FLDCE_BF16 ? (size_t)C * p->cfg.D * 4 : 0);
     const bool acc = L.nchunks > 1 && !dw_out_fp32(p);
     L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
     L.total = off;
@@ -263,7 +289,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
 
     CUtensorMap mW_k, mW_mn;
     if (bf16 && N > 0) {
-        if (!make_map(&mW_k, W, D, V, D, 64, kBN)) return FLDCE_ERR_CUDA;
+        if (!make_map(&mW_k, W, D, V, D, 64, 128)) return FLDCE_ERR_CUDA;
         if (backward && !make_map(&mW_mn, W, D, V, D, 64, 64)) return FLDCE_ERR_CUDA;
     }
 
@@ -288,8 +314,8 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         if (bf16) {
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
             if (!make_map(&mH_k, Hc, D, rows, D, 64, 128)) return FLDCE_ERR_CUDA;
-            FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, lp, &cnt->dev_err,
-                                                   dev.sms, st)));
+            FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, 1, lp,
+                                                   &cnt->dev_err, dev.sms, st)));
         } else {
             const float* Hc = static_cast<const float*>(H) + r0 * D;
             SimtLse e{lp};
@@ -326,21 +352,22 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         prof_mark(h, PK_MERGE, st);
         if (!backward) continue;
 
-        const int mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : (ci + 1 < L.nchunks || fp32_dw ? 2 : 3));
+        // dW: one chunk writes the output directly; several chunks store, then
+        // reduce-add, fp32 partial sums (into dW itself when it is fp32).
+        const int simt_mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : 2);
         if (bf16) {
             __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(ws + L.G);
             GEpi::Params gp;
+            if (!make_store_map(&gp.gmap, G, V, rows, h->Vpad, 2)) return FLDCE_ERR_CUDA;
             gp.c = c;
             gp.V = V;
-            gp.ldg = h->Vpad;
             gp.rows = rows;
             gp.lse2 = row_lse2;
             gp.gcoef = row_gcoef;
             gp.ycol = row_y;
             gp.eps_over_V = eps / (float)V;
             gp.one_minus_eps = 1.f - eps;
-            gp.G = G;
-            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, gp, &cnt->dev_err,
+            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, 1, gp, &cnt->dev_err,
                                                  dev.sms, st)));
             prof_mark(h, PK_G, st);
             if (!make_map(&mG_k, G, V, rows, h->Vpad, 64, 128)) return FLDCE_ERR_CUDA;
@@ -348,28 +375,50 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
             if (!make_map(&mH_mn, Hc, D, rows, D, 64, 64)) return FLDCE_ERR_CUDA;
 
+            // dH = G W (K = V).  When one pass over the tiles leaves many SMs
+            // idle in its last round, the vocabulary is split in two halves
+            // whose fp32 partials are reduce-added into a zeroed buffer (two
+            // addends: the sum does not depend on their order).
+            const int pairs = std::max(1, dev.sms / 2);
+            const int64_t dh_tiles = cdiv(rows, CfgKM::PAIR_M) * cdiv(D, CfgKM::BN);
+            const bool dh_split = cdiv(V, CfgKM::BK) >= 8 &&
+                                  wave_efficiency(2 * dh_tiles, pairs) >
+                                      wave_efficiency(dh_tiles, pairs) + 0.03;
             StoreEpi::Params hp;
-            hp.rows = rows;
-            hp.cols = D;
-            hp.ldo = D;
-            hp.out = static_cast<__nv_bfloat16*>(dH) + r0 * D;
-            hp.ws = nullptr;
-            hp.mode = 0;
-            hp.out_fp32 = 0;
-            FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1, hp,
-                                                     &cnt->dev_err, dev.sms, st)));
+            float* dh_acc = reinterpret_cast<float*>(ws + L.dh_acc);
+            void* dHc = static_cast<__nv_bfloat16*>(dH) + r0 * D;
+            if (dh_split) {
+                FLDCE_CUDA(cudaMemsetAsync(dh_acc, 0, (size_t)rows * D * 4, st));
+                if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
+                hp.mode = WS_ADD;
+            } else {
+                if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
+                hp.mode = OUT_BF16;
+            }
+            FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1,
+                                                     dh_split ? 2 : 1, hp, &cnt->dev_err,
+                                                     dev.sms, st)));
             prof_mark(h, PK_DH, st);
+            if (dh_split) {
+                FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
+                prof_mark(h, PK_CONVERT, st);
+            }
+
             StoreEpi::Params wp;
-            wp.rows = (int)V;
-            wp.cols = D;
-            wp.ldo = D;
-            wp.out = dW;
-            wp.ws = dw_ws;
-            wp.mode = mode;
-            wp.out_fp32 = fp32_dw ? 1 : 0;
-            FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, wp,
+            if (L.nchunks == 1 && !fp32_dw) {
+                if (!make_store_map(&wp.omap, dW, D, V, D, 2)) return FLDCE_ERR_CUDA;
+                wp.mode = OUT_BF16;
+            } else {
+                if (!make_store_map(&wp.omap, dw_ws, D, V, D, 4)) return FLDCE_ERR_CUDA;
+                wp.mode = ci == 0 ? WS_STORE : WS_ADD;
+            }
+            FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, 1, wp,
                                                      &cnt->dev_err, dev.sms, st)));
             prof_mark(h, PK_DW, st);
+            if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {
+                FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, dev.sms, st));
+                prof_mark(h, PK_CONVERT, st);
+            }
         } else {
             float* G = reinterpret_cast<float*>(ws + L.G);
             const float* Hc = static_cast<const float*>(H) + r0 * D;
@@ -381,7 +430,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             FLDCE_CUDA(launch_simt(G, h->Vpad, 1, static_cast<const float*>(W), 1, D, rows, D,
                                    (int)V, hs, st));
             prof_mark(h, PK_DH, st);
-            SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, mode == 3 ? 2 : mode};
+            SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, simt_mode};
             FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
             prof_mark(h, PK_DW, st);
         }
@@ -502,7 +551,7 @@ int fldce_forward(fldce_handle h, const void* H, const void* W, const int64_t* t
 int fldce_profile_begin(fldce_handle h, int max_calls) {
     if (h == nullptr || max_calls <= 0) return FLDCE_ERR_INVALID_ARG;
     const int64_t chunks = cdiv(h->cfg.max_N, h->chunk);
-    const size_t need = (size_t)max_calls * (size_t)(3 + 5 * chunks);
+    const size_t need = (size_t)max_calls * (size_t)(4 + 6 * chunks);
     while (h->ev.size() < need) {
         cudaEvent_t e;
         if (cudaEventCreate(&e) != cudaSuccess) return FLDCE_ERR_CUDA;
@@ -539,7 +588,8 @@ int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches) {
 
 const char* fldce_profile_kind_name(int kind) {
     static const char* names[FLDCE_PROF_KINDS] = {"count_targets", "lse_sweep", "merge",
-                                                  "g_sweep", "dh_gemm", "dw_gemm", "finish"};
+                                                  "g_sweep", "dh_gemm", "dw_gemm", "finish",
+                                                  "convert"};
     return (kind >= 0 && kind < FLDCE_PROF_KINDS) ? names[kind] : nullptr;
 }
 

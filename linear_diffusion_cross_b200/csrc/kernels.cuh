@@ -26,8 +26,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Walk the eight 32-column chunks of this thread's accumulator row with the
+// next chunk's TMEM load in flight while the current one is processed;
+// `f(r, j)` sees chunk j.  The accumulator is released to the MMA warp as
+// soon as the last chunk has landed in registers.
+template <class F>
+__device__ __forceinline__ void for_each_chunk(const AccRow& acc, F&& f) {
+    uint32_t ra[32], rb[32];
+    acc.load(0, ra);
+#pragma unroll 1
+    for (int j = 0; j < 8; j += 2) {
+        acc.issue(j + 1, rb);
+        f(ra, j);
+        acc.wait(rb);
+        if (j + 2 < 8) acc.issue(j + 2, ra); else acc.release();
+        f(rb, j + 1);
+        if (j + 2 < 8) acc.wait(ra);
+    }
+}
+
 // ======================================================================
-// Epilogue 1 (sweep 1): per-row partial logsumexp of one vocab tile.
+// Epilogue 1 (sweep 1): per-row partial logsumexp of one 256-wide vocab tile.
 // logsumexp_fwd_kernel keeps one (max, log-sum-exp) per row and vocab block;
 // here each (row, vocab tile) keeps (m2, l) plus, when asked, the sum of the
 // raw logits (label smoothing), the tile argmax, and the target logit when
@@ -47,46 +66,44 @@ struct LseEpi {
         float* zy;               // [ld_part] target logit z[n, y_n]
     };
 
-    template <int BN>
-    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
-                                               const AccRow& acc) {
-        const int m = mt * 128 + row;
-        const int64_t n0 = (int64_t)nt * BN;
+    template <class Cfg>
+    static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
+                                               const AccRow& acc, Stager&) {
+        const int m = t.row0 + t.row;
+        const int64_t n0 = t.col0;
+        const int nt = (int)(n0 / Cfg::BN);
         const bool live = m < p.rows;
         int yrel = -1;
         if (live) {
             const int64_t y = p.target[m];
-            if (y >= n0 && y < n0 + BN && y < p.V) yrel = (int)(y - n0);
+            if (y >= n0 && y < n0 + Cfg::BN && y < p.V) yrel = (int)(y - n0);
         }
-        const int ncols = (int)((p.V - n0) < BN ? (p.V - n0) : BN);
+        const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
+        const bool want_am = p.part_am != nullptr, want_sz = p.part_sz != nullptr;
         float mx = -CUDART_INF_F, l = 0.f, sz = 0.f, zyv = 0.f, amv = -CUDART_INF_F;
         int am = 0;
-#pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
-            uint32_t r[32];
-            acc.load(j, r);
-            if (j == BN / 32 - 1) acc.release();
-            float t[32];
+        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
+            float tv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) t[i] = __uint_as_float(r[i]) * p.c;
+            for (int i = 0; i < 32; ++i) tv[i] = __uint_as_float(r[i]) * p.c;
             if (32 * j + 32 > ncols) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (32 * j + i >= ncols) t[i] = -CUDART_INF_F;
+                    if (32 * j + i >= ncols) tv[i] = -CUDART_INF_F;
             }
-            float cm0 = fmaxf(t[0], t[1]), cm1 = fmaxf(t[2], t[3]);
+            float cm0 = fmaxf(tv[0], tv[1]), cm1 = fmaxf(tv[2], tv[3]);
 #pragma unroll
             for (int i = 4; i < 32; i += 4) {
-                cm0 = fmaxf(cm0, fmaxf(t[i], t[i + 1]));
-                cm1 = fmaxf(cm1, fmaxf(t[i + 2], t[i + 3]));
+                cm0 = fmaxf(cm0, fmaxf(tv[i], tv[i + 1]));
+                cm1 = fmaxf(cm1, fmaxf(tv[i + 2], tv[i + 3]));
             }
             const float nm = fmaxf(mx, fmaxf(cm0, cm1));
-            if (p.part_am != nullptr) {
+            if (want_am) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (t[i] > amv) { amv = t[i]; am = 32 * j + i; }
+                    if (tv[i] > amv) { amv = tv[i]; am = 32 * j + i; }
             }
-            if (p.part_sz != nullptr) {
+            if (want_sz) {
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
@@ -103,70 +120,89 @@ struct LseEpi {
             float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-                e0 += ex2(t[i] - nm);
-                e1 += ex2(t[i + 1] - nm);
-                e2 += ex2(t[i + 2] - nm);
-                e3 += ex2(t[i + 3] - nm);
+                e0 += ex2(tv[i] - nm);
+                e1 += ex2(tv[i + 1] - nm);
+                e2 += ex2(tv[i + 2] - nm);
+                e3 += ex2(tv[i + 3] - nm);
             }
             l = l * ex2(mx - nm) + ((e0 + e1) + (e2 + e3));
             mx = nm;
-        }
+        });
         if (live) {
             const size_t o = (size_t)nt * p.ld_part + m;
             p.part_ml[o] = make_float2(mx, l);
-            if (p.part_sz != nullptr) p.part_sz[o] = sz;
-            if (p.part_am != nullptr) p.part_am[o] = (int32_t)(n0 + am);
+            if (want_sz) p.part_sz[o] = sz;
+            if (want_am) p.part_am[o] = (int32_t)(n0 + am);
             if (yrel >= 0) p.zy[m] = zyv * p.s;
         }
     }
 };
+
+// Pack 16 fp32 values of r (from r[off]) as bf16 into two 16-byte chunks.
+__device__ __forceinline__ void pack16(const float* v, uint4& a, uint4& b) {
+    a.x = pack_bf16x2(v[0], v[1]);
+    a.y = pack_bf16x2(v[2], v[3]);
+    a.z = pack_bf16x2(v[4], v[5]);
+    a.w = pack_bf16x2(v[6], v[7]);
+    b.x = pack_bf16x2(v[8], v[9]);
+    b.y = pack_bf16x2(v[10], v[11]);
+    b.z = pack_bf16x2(v[12], v[13]);
+    b.w = pack_bf16x2(v[14], v[15]);
+}
+
+// Stage 32 bf16 values (chunk j of the row) into half of the 128-byte row
+// segment; chunk pairs (2 jj, 2 jj + 1) form one 64-column store box.
+__device__ __forceinline__ void stage_bf16_half(Stager& st, int j, const float (&v)[32]) {
+    uint4 a, b, c, d;
+    pack16(v, a, b);
+    pack16(v + 16, c, d);
+    const int base = (j & 1) * 4;
+    st.put(base + 0, a);
+    st.put(base + 1, b);
+    st.put(base + 2, c);
+    st.put(base + 3, d);
+}
 
 // ======================================================================
 // Epilogue 2 (sweep 2): the gradient of the logits, rounded once to bf16.
 // cross_entropy_kernel steps 5-6 and the backward's grad_out:
 //   G = gcoef * (2^(t - lse2) - eps/V) - gcoef * (1 - eps) [v = y],
 //   gcoef = g s / (p T), exactly 0 for ignored tokens and columns >= V.
+// G leaves through the stager in 32-row x 64-column boxes (TMA store; the
+// store map's extent clips rows past the chunk and columns past V).
 // ======================================================================
 struct GEpi {
     struct Params {
+        CUtensorMap gmap;        // G [rows, V] bf16, box 64 x 32, 128B swizzle
         float c;
         int64_t V;
-        int64_t ldg;             // row stride of G in elements (multiple of 8)
         int rows;
         const float* lse2;       // [chunk] lse in base-2 units
         const float* gcoef;      // [chunk]
         const int32_t* ycol;     // [chunk] validated target or -1
         float eps_over_V;
         float one_minus_eps;
-        __nv_bfloat16* G;        // [chunk][ldg]
     };
 
-    template <int BN>
-    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
-                                               const AccRow& acc) {
-        const int m = mt * 128 + row;
-        const int64_t n0 = (int64_t)nt * BN;
-        const bool live = m < p.rows;
+    template <class Cfg>
+    static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
+                                               const AccRow& acc, Stager& st) {
+        const int m = t.row0 + t.row;
+        const int64_t n0 = t.col0;
         float gc = 0.f, L2 = 0.f;
         int yrel = -1;
-        if (live) {
+        if (m < p.rows) {
             gc = p.gcoef[m];
             if (gc != 0.f) {
                 L2 = p.lse2[m];
                 const int y = p.ycol[m];
-                if (y >= n0 && y < n0 + BN) yrel = (int)(y - n0);
+                if (y >= n0 && y < n0 + Cfg::BN) yrel = (int)(y - n0);
             }
         }
         const float base = gc * p.eps_over_V;
         const float tcorr = gc * p.one_minus_eps;
-        const int ncols = (int)((p.V - n0) < BN ? (p.V - n0) : BN);
-        const int scols = (int)((p.ldg - n0) < BN ? (p.ldg - n0) : BN);
-        __nv_bfloat16* grow = p.G + (size_t)(live ? m : 0) * p.ldg + n0;
-#pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
-            uint32_t r[32];
-            acc.load(j, r);
-            if (j == BN / 32 - 1) acc.release();
+        const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
+        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
             float g[32];
             if (gc != 0.f) {
 #pragma unroll
@@ -186,83 +222,49 @@ struct GEpi {
                 for (int i = 0; i < 32; ++i)
                     if (32 * j + i >= ncols) g[i] = 0.f;
             }
-            if (live) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (32 * j + 8 * q < scols) {
-                        uint4 v;
-                        v.x = pack_bf16x2(g[8 * q + 0], g[8 * q + 1]);
-                        v.y = pack_bf16x2(g[8 * q + 2], g[8 * q + 3]);
-                        v.z = pack_bf16x2(g[8 * q + 4], g[8 * q + 5]);
-                        v.w = pack_bf16x2(g[8 * q + 6], g[8 * q + 7]);
-                        *reinterpret_cast<uint4*>(grow + 32 * j + 8 * q) = v;
-                    }
-                }
-            }
-        }
+            if ((j & 1) == 0) st.acquire();
+            stage_bf16_half(st, j, g);
+            if (j & 1) st.flush(&p.gmap, (int)(n0 + 32 * (j - 1)), t.row0 + 32 * t.q, false);
+        });
     }
 };
 
 // ======================================================================
-// Epilogue 3: dH / dW tiles.  mode 0: out = acc; 1: ws = acc; 2: ws += acc;
-// 3: out = ws + acc (fp32 workspace ws carries dW across token chunks).
+// Epilogue 3: dH / dW tiles.
+//   OUT_BF16: bf16 output, 64-column boxes, TMA store;
+//   WS_STORE / WS_ADD: fp32 32-column boxes, TMA store or TMA reduce-add
+//   (dW accumulated over token chunks; dH split over two vocab halves).
 // ======================================================================
+enum StoreMode { OUT_BF16 = 0, WS_STORE = 1, WS_ADD = 2 };
+
 struct StoreEpi {
     struct Params {
-        int rows;                // valid output rows
-        int64_t cols;            // valid output columns
-        int64_t ldo;             // row stride of out / ws (elements)
-        void* out;               // bf16 or fp32
-        float* ws;               // fp32 accumulator (modes 1-3)
+        CUtensorMap omap;        // bf16 [rows, cols] box 64 x 32, or fp32 box 32 x 32
         int mode;
-        int out_fp32;
     };
 
-    template <int BN>
-    static __device__ __forceinline__ void run(const Params& p, int mt, int nt, int row,
-                                               const AccRow& acc) {
-        const int m = mt * 128 + row;
-        const int64_t n0 = (int64_t)nt * BN;
-        const bool live = m < p.rows;
-        const size_t rbase = (size_t)(live ? m : 0) * p.ldo + n0;
-#pragma unroll 1
-        for (int j = 0; j < BN / 32; ++j) {
-            uint32_t r[32];
-            acc.load(j, r);
-            if (j == BN / 32 - 1) acc.release();
-            if (!live) continue;
-            float v[32];
+    template <class Cfg>
+    static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
+                                               const AccRow& acc, Stager& st) {
+        const int64_t n0 = t.col0;
+        const int y = t.row0 + 32 * t.q;
+        const int mode = p.mode;
+        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
+            if (mode == OUT_BF16) {
+                float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                if ((j & 1) == 0) st.acquire();
+                stage_bf16_half(st, j, v);
+                if (j & 1) st.flush(&p.omap, (int)(n0 + 32 * (j - 1)), y, false);
+            } else {
+                st.acquire();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int64_t col = n0 + 32 * j + 8 * q;
-                if (col >= p.cols) continue;
-                const size_t o = rbase + 32 * j + 8 * q;
-                float* x = v + 8 * q;
-                if (p.mode >= 2) {
-                    const float4 a = *reinterpret_cast<const float4*>(p.ws + o);
-                    const float4 b = *reinterpret_cast<const float4*>(p.ws + o + 4);
-                    x[0] += a.x; x[1] += a.y; x[2] += a.z; x[3] += a.w;
-                    x[4] += b.x; x[5] += b.y; x[6] += b.z; x[7] += b.w;
-                }
-                if (p.mode == 1 || p.mode == 2) {
-                    *reinterpret_cast<float4*>(p.ws + o) = make_float4(x[0], x[1], x[2], x[3]);
-                    *reinterpret_cast<float4*>(p.ws + o + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                } else if (p.out_fp32) {
-                    float* out = reinterpret_cast<float*>(p.out) + o;
-                    *reinterpret_cast<float4*>(out) = make_float4(x[0], x[1], x[2], x[3]);
-                    *reinterpret_cast<float4*>(out + 4) = make_float4(x[4], x[5], x[6], x[7]);
-                } else {
-                    uint4 w;
-                    w.x = pack_bf16x2(x[0], x[1]);
-                    w.y = pack_bf16x2(x[2], x[3]);
-                    w.z = pack_bf16x2(x[4], x[5]);
-                    w.w = pack_bf16x2(x[6], x[7]);
-                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o) = w;
-                }
+                for (int c = 0; c < 8; ++c)
+                    st.put(c, make_uint4(r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]));
+                st.flush(&p.omap, (int)(n0 + 32 * j), y, mode == WS_ADD);
             }
-        }
+        });
     }
 };
 
@@ -388,6 +390,22 @@ __global__ void k_finish(const float* __restrict__ loss_tok, int64_t N, const Co
             err_count[0] = cnt->n_err;
             err_count[1] = cnt->dev_err;
         }
+    }
+}
+
+// fp32 -> bf16 (round to nearest even), 8 elements per thread and step.
+__global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                              int64_t n8) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+        const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+        uint4 w;
+        w.x = pack_bf16x2(a.x, a.y);
+        w.y = pack_bf16x2(a.z, a.w);
+        w.z = pack_bf16x2(b.x, b.y);
+        w.w = pack_bf16x2(b.z, b.w);
+        reinterpret_cast<uint4*>(dst)[i] = w;
     }
 }
 

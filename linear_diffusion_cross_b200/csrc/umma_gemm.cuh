@@ -1,27 +1,36 @@
-// umma_gemm.cuh -- persistent tcgen05 GEMM for sm_100a with pluggable epilogues.
+// umma_gemm.cuh -- persistent tcgen05 GEMM on CTA pairs for sm_100a, with
+// pluggable epilogues.
 //
 // D[m, n] = sum_k A[m, k] * B[n, k] over bf16 operands with an fp32
-// accumulator that lives in tensor memory (TMEM).  One CTA per SM walks a
-// static round-robin list of BM x BN output tiles:
+// accumulator in tensor memory (TMEM).  Work is cut into 256 x 256 output
+// tiles (optionally also into K splits).  Each tile belongs to a cluster of
+// two CTAs on neighbouring SMs that issue one tcgen05.mma.cta_group::2 per
+// K step of 16: CTA r of the pair holds rows [128 r, 128 r + 128) of the A
+// tile and of the B tile in its shared memory, and receives rows
+// [128 r, 128 r + 128) of the 256 x 256 accumulator in its TMEM.  Each SM
+// therefore streams 32 KB of operands per 64-wide K step instead of the
+// 48 KB a single-CTA 128 x 256 tile needs, a third less L2 -> SM traffic
+// for the same tensor work.
 //
-//   warp 0      TMA producer: 128B-swizzled tiles of A and B into a
-//               STAGES-deep shared-memory ring (full/empty mbarriers).
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
-//               K=16) into one of two TMEM accumulators, commits the ring
-//               slot back to the producer and the finished accumulator to
-//               the epilogue.
-//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane),
-//               reads it 32 columns at a time with tcgen05.ld and hands the
-//               values to the epilogue functor; the accumulator is released
-//               as soon as it is read, so the next tile's MMAs overlap the
-//               current tile's epilogue.
+// Roles (192 threads per CTA):
+//   warp 0      TMA producer (both CTAs): loads this CTA's halves into a
+//               STAGES-deep ring; completion is counted on the pair leader's
+//               "full" mbarrier, which expects the bytes of both CTAs.
+//   warp 1      MMA issuer (leader CTA only issues; both allocate TMEM):
+//               waits for a full stage, issues four M=256 N=256 K=16 MMAs and
+//               commits the stage back to both producers (multicast commit),
+//               then commits a finished accumulator to both epilogues.
+//   warps 2..5  epilogue (both CTAs): one accumulator row per thread, read
+//               with tcgen05.ld while the next tile's MMAs run into the other
+//               of the two TMEM accumulators; output tiles leave through a
+//               per-warp 128B-swizzled staging buffer and TMA bulk stores (or
+//               bulk reduce-adds).
 //
-// Operands may be K-major (K contiguous) or MN-major (M/N contiguous); both
-// are consumed straight from their row-major HBM layout through the TMA
-// tensor map, so no transposed copy of any operand is ever made.
-//
-// Every mbarrier wait is bounded by global time; on time-out the CTA records
-// FLDCE_DEV_ERR_TIMEOUT in `err`, stops issuing work and frees its TMEM.
+// Operands are consumed K-major or MN-major straight from row-major HBM
+// through the tensor maps; no transposed copy of any operand is made.  Loads
+// carry no cluster multicast.  Every mbarrier wait is bounded by global time;
+// on time-out the CTA records FLDCE_DEV_ERR_TIMEOUT, stops issuing work and
+// frees its TMEM.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -35,76 +44,124 @@ constexpr int kGemmThreads = 192;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
 constexpr int32_t FLDCE_DEV_ERR_TIMEOUT = 1;
 
-template <int BN_, int STAGES_, bool A_MN_, bool B_MN_>
+template <int STAGES_, bool A_MN_, bool B_MN_>
 struct GemmCfg {
-    static constexpr int BM = 128;
-    static constexpr int BN = BN_;
-    static constexpr int BK = 64;                 // one 128-byte swizzle span of bf16
+    static constexpr int BM = 128;                 // accumulator rows per CTA
+    static constexpr int PAIR_M = 256;             // rows of a pair tile
+    static constexpr int BN = 256;                 // columns of a tile
+    static constexpr int BN_HALF = 128;            // B rows held per CTA
+    static constexpr int BK = 64;                  // one 128-byte swizzle span of bf16
     static constexpr int STAGES = STAGES_;
     static constexpr bool A_MN = A_MN_;
     static constexpr bool B_MN = B_MN_;
     static constexpr uint32_t A_BYTES = BM * BK * 2;
-    static constexpr uint32_t B_BYTES = BN * BK * 2;
+    static constexpr uint32_t B_BYTES = BN_HALF * BK * 2;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+    static constexpr uint32_t EPI_BUF_BYTES = 32 * 128;       // 32 rows x 128 B
+    static constexpr uint32_t EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
     static constexpr uint32_t BAR_BYTES = 256;
-    static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
-    static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, A_MN, B_MN);
-    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-    static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+    static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+    static constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_M, BN, A_MN, B_MN);
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 struct GemmGeom {
-    int tiles_m;
-    int tiles_n;
+    int tiles_m;          // ceil(M / 256)
+    int tiles_n;          // ceil(N / 256)
     int k_iters;          // ceil(K / 64)
-    int num_tiles;
+    int k_splits;         // K ranges per tile (1 or 2)
+    int num_tiles;        // tiles_m * tiles_n
     int n_fastest;        // 1: consecutive tiles walk n first (share the A panel)
 };
 
-__device__ __forceinline__ void tile_coords(const GemmGeom& g, int tile, int& mt, int& nt) {
-    if (g.n_fastest) {
-        nt = tile % g.tiles_n;
-        mt = tile / g.tiles_n;
-    } else {
-        mt = tile % g.tiles_m;
-        nt = tile / g.tiles_m;
-    }
-}
+// Where the current tile of this thread sits.
+struct TileCtx {
+    int row0;             // output row of TMEM lane 0 of this CTA
+    int64_t col0;         // first output column of the tile
+    int split;            // K split index
+    int row;              // this thread's accumulator row (TMEM lane), 0..127
+    int q;                // warp quadrant: rows [32 q, 32 q + 32)
+    int lane;
+};
 
 // Per-thread view of one accumulator row handed to an epilogue functor.
 struct AccRow {
     uint32_t taddr;       // TMEM address of this thread's lane, column 0 of the tile
-    uint32_t tempty_bar;  // mbarrier to arrive on once every column has been read
+    uint32_t tempty_bar;  // leader's accumulator-empty mbarrier (cluster address)
     int lane;
 
-    // Load columns [32*j, 32*j + 32) of the row (waits for completion).
-    __device__ __forceinline__ void load(int j, uint32_t (&r)[32]) const {
+    // Issue loads of columns [32 j, 32 j + 32); complete them with wait().
+    __device__ __forceinline__ void issue(int j, uint32_t (&r)[32]) const {
         tmem_ld_32x32b_x32(taddr + (uint32_t)(32 * j), r);
-        tmem_ld_wait();
     }
-    // Hand the accumulator back to the MMA warp (one arrive per warp).
+    __device__ __forceinline__ void wait(uint32_t (&r)[32]) const { tmem_ld_wait_regs(r); }
+    __device__ __forceinline__ void load(int j, uint32_t (&r)[32]) const {
+        issue(j, r);
+        wait(r);
+    }
+    // Hand the accumulator back to the pair's MMA warp (one arrive per warp).
     __device__ __forceinline__ void release() const {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar);
+        if (lane == 0) mbar_arrive_cluster(tempty_bar);
+    }
+};
+
+// One warp's two 32-row x 128-byte staging buffers and its TMA stores.  Row
+// r's 16-byte chunk c lives at r*128 + ((c ^ (r & 7)) * 16): the 128-byte
+// swizzle the store tensor maps use, which also keeps the 32 lanes' writes
+// free of bank conflicts.
+struct Stager {
+    uint32_t buf0;
+    int lane;
+    int phase;
+
+    __device__ __forceinline__ uint32_t cur() const { return buf0 + (uint32_t)phase * 4096u; }
+    // Make sure the buffer about to be written is no longer read by a store.
+    __device__ __forceinline__ void acquire() {
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+    }
+    __device__ __forceinline__ void put(int c, uint4 v) {
+        st_shared_v4(cur() + (uint32_t)lane * 128u + (uint32_t)((c ^ (lane & 7)) << 4), v);
+    }
+    // Store (or reduce-add) the staged 32 x 128 B box at (x, y) of `m`.
+    __device__ __forceinline__ void flush(const CUtensorMap* m, int x, int y, bool add) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            if (add) tma_reduce_add_2d(m, cur(), x, y);
+            else tma_store_2d(m, cur(), x, y);
+            bulk_commit_group();
+        }
+        phase ^= 1;
+    }
+    __device__ __forceinline__ void drain() {
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 };
 
 template <class Cfg, class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmGeom geom, const typename Epi::Params ep, int32_t* err) {
+                 const GemmGeom geom, const __grid_constant__ typename Epi::Params ep,
+                 int32_t* err) {
     constexpr int S = Cfg::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::STAGE_BYTES);
+    uint8_t* epi_smem = smem + S * Cfg::STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + Cfg::EPI_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();          // 0 = pair leader
+    const uint32_t pair = cluster_id_x();
+    const uint32_t npairs = cluster_count_x();
     const uint32_t sbase = smem_u32(smem);
     auto full_bar = [&](int s) { return smem_u32(bars + s); };
     auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
@@ -118,7 +175,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);
+            mbar_init(tempty_bar(b), 8);       // 4 epilogue warps x 2 CTAs
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -126,113 +183,159 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                            // the peer's barriers exist before use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const int units = geom.num_tiles * geom.k_splits;
+    const int kps = (geom.k_iters + geom.k_splits - 1) / geom.k_splits;
 
     auto fail = [&]() {
         *abort_flag = 1;
         if (lane == 0) atomicOr(err, FLDCE_DEV_ERR_TIMEOUT);
     };
+    auto unit_coords = [&](int u, int& mt, int& nt, int& split, int& k0, int& k1) {
+        split = u / geom.num_tiles;
+        const int tile = u - split * geom.num_tiles;
+        if (geom.n_fastest) {
+            nt = tile % geom.tiles_n;
+            mt = tile / geom.tiles_n;
+        } else {
+            mt = tile % geom.tiles_m;
+            nt = tile / geom.tiles_m;
+        }
+        k0 = split * kps;
+        k1 = min(geom.k_iters, k0 + kps);
+    };
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         const uint64_t pol = l2_policy_evict_normal();
+        const uint32_t lead_full0 = mapa_shared(full_bar(0), 0);
         uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < geom.num_tiles && !*abort_flag; tile += gridDim.x) {
-            int mt, nt;
-            tile_coords(geom, tile, mt, nt);
-            for (int k = 0; k < geom.k_iters; ++k, ++it) {
+        bool ok = true;
+        for (int u = pair; ok && u < units && !*abort_flag; u += npairs) {
+            int mt, nt, split, k0, k1;
+            unit_coords(u, mt, nt, split, k0, k1);
+            const int arow = mt * Cfg::PAIR_M + (int)rank * Cfg::BM;
+            const int brow = nt * Cfg::BN + (int)rank * Cfg::BN_HALF;
+            for (int k = k0; k < k1; ++k, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1u;
-                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs)) { fail(); break; }
+                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, kWaitLimitNs)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
                 if (lane == 0) {
                     const uint32_t sa = sbase + s * Cfg::STAGE_BYTES;
                     const uint32_t sb = sa + Cfg::A_BYTES;
-                    mbar_arrive_expect_tx(full_bar(s), Cfg::STAGE_BYTES);
+                    const uint32_t fb = lead_full0 + 8u * (uint32_t)s;
+                    if (rank == 0) mbar_arrive_expect_tx(full_bar(s), 2 * Cfg::STAGE_BYTES);
                     if (Cfg::A_MN) {
 #pragma unroll
                         for (int j = 0; j < Cfg::BM / 64; ++j)
-                            tma_load_2d(sa + j * 8192, &tmA, full_bar(s), mt * Cfg::BM + 64 * j,
-                                        k * Cfg::BK, pol);
+                            tma_load_2d_pair(sa + j * 8192, &tmA, fb, arow + 64 * j, k * Cfg::BK,
+                                             pol);
                     } else {
-                        tma_load_2d(sa, &tmA, full_bar(s), k * Cfg::BK, mt * Cfg::BM, pol);
+                        tma_load_2d_pair(sa, &tmA, fb, k * Cfg::BK, arow, pol);
                     }
                     if (Cfg::B_MN) {
 #pragma unroll
-                        for (int j = 0; j < Cfg::BN / 64; ++j)
-                            tma_load_2d(sb + j * 8192, &tmB, full_bar(s), nt * Cfg::BN + 64 * j,
-                                        k * Cfg::BK, pol);
+                        for (int j = 0; j < Cfg::BN_HALF / 64; ++j)
+                            tma_load_2d_pair(sb + j * 8192, &tmB, fb, brow + 64 * j, k * Cfg::BK,
+                                             pol);
                     } else {
-                        tma_load_2d(sb, &tmB, full_bar(s), k * Cfg::BK, nt * Cfg::BN, pol);
+                        tma_load_2d_pair(sb, &tmB, fb, k * Cfg::BK, brow, pol);
                     }
                 }
                 __syncwarp();
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        uint32_t it = 0, lt = 0;
-        for (int tile = blockIdx.x; tile < geom.num_tiles && !*abort_flag;
-             tile += gridDim.x, ++lt) {
-            const int b = lt & 1;
-            const uint32_t use = lt >> 1;
-            if (!mbar_wait_bounded(tempty_bar(b), (use & 1u) ^ 1u, kWaitLimitNs)) { fail(); break; }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(b * Cfg::BN);
-            bool ok = true;
-            for (int k = 0; k < geom.k_iters; ++k, ++it) {
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1u;
-                if (!mbar_wait_bounded(full_bar(s), ph, kWaitLimitNs)) { fail(); ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t sa = sbase + s * Cfg::STAGE_BYTES;
-                    const uint32_t sb = sa + Cfg::A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
-                        const uint64_t ad = Cfg::A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
-                                                      : smem_desc_sw128(sa + kk * 32, 16, 1024);
-                        const uint64_t bd = Cfg::B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
-                        tc_mma_f16(d_tmem, ad, bd, Cfg::IDESC, (k | kk) != 0 ? 1u : 0u);
-                    }
-                    tc_commit(empty_bar(s));
+        // ------------------------------------------------ MMA issuer (leader)
+        if (rank == 0) {
+            uint32_t it = 0, lt = 0;
+            for (int u = pair; u < units && !*abort_flag; u += npairs, ++lt) {
+                int mt, nt, split, k0, k1;
+                unit_coords(u, mt, nt, split, k0, k1);
+                const int b = lt & 1;
+                const uint32_t use = lt >> 1;
+                if (!mbar_wait_bounded(tempty_bar(b), (use & 1u) ^ 1u, kWaitLimitNs)) {
+                    fail();
+                    break;
                 }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * Cfg::BN);
+                bool ok = true;
+                for (int k = k0; k < k1; ++k, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait_bounded(full_bar(s), ph, kWaitLimitNs)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t sa = sbase + s * Cfg::STAGE_BYTES;
+                        const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < Cfg::BK / 16; ++kk) {
+                            const uint64_t ad =
+                                Cfg::A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sa + kk * 32, 16, 1024);
+                            const uint64_t bd =
+                                Cfg::B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
+                            tc_mma_f16_pair(d_tmem, ad, bd, Cfg::IDESC,
+                                            (k > k0 || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit_pair_mc(empty_bar(s), 0x3);
+                    }
+                    __syncwarp();
+                }
+                if (!ok) break;
+                if (lane == 0) tc_commit_pair_mc(tfull_bar(b), 0x3);
                 __syncwarp();
             }
-            if (!ok) break;
-            if (lane == 0) tc_commit(tfull_bar(b));
-            __syncwarp();
         }
     } else {
-        // ------------------------------------------------ epilogue
+        // ------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const int row = q * 32 + lane;          // accumulator row owned by this thread
+        Stager st{smem_u32(epi_smem) + (uint32_t)(q * 2) * Cfg::EPI_BUF_BYTES, lane, 0};
+        const uint32_t lead_tempty0 = mapa_shared(tempty_bar(0), 0);
         uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < geom.num_tiles && !*abort_flag;
-             tile += gridDim.x, ++lt) {
+        for (int u = pair; u < units && !*abort_flag; u += npairs, ++lt) {
+            int mt, nt, split, k0, k1;
+            unit_coords(u, mt, nt, split, k0, k1);
             const int b = lt & 1;
             const uint32_t use = lt >> 1;
-            if (!mbar_wait_bounded(tfull_bar(b), use & 1u, kWaitLimitNs)) { fail(); break; }
+            if (!mbar_wait_bounded(tfull_bar(b), use & 1u, kWaitLimitNs)) {
+                fail();
+                break;
+            }
             tc_fence_after();
-            int mt, nt;
-            tile_coords(geom, tile, mt, nt);
+            TileCtx t{mt * Cfg::PAIR_M + (int)rank * Cfg::BM, (int64_t)nt * Cfg::BN, split, row,
+                      q, lane};
             AccRow acc{tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * Cfg::BN),
-                       tempty_bar(b), lane};
-            Epi::template run<Cfg::BN>(ep, mt, nt, row, acc);
+                       lead_tempty0 + 8u * (uint32_t)b, lane};
+            Epi::template run<Cfg>(ep, t, acc, st);
         }
+        st.drain();
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();            // every MMA of the pair has completed and been read
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
     }
 }
 
