@@ -298,12 +298,21 @@ def main():
         chunks = -(-N // B.fldce_chunk_size(plan.handle))
         fl_launch = 2.0 * N * D * V / chunks
         ach = fl_launch / (dom_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": dom, "achieved": ach,
-                "peak": peaks[peak_key], "unit": "TFLOP/s", "frac": ach / peaks[peak_key],
-                "peak_source": f"{peaks_src} {peak_key}",
-                "frac_of_burst": ach / peaks["bf16_tflops"],
-                "flops_per_launch": fl_launch, "ms_per_launch": dom_ms,
-                "traffic": traffic_for(dom, args.workload)}
+        if wl.H.dtype == torch.bfloat16:
+            roof = {"bound": "tensor", "kernel": dom, "achieved": ach,
+                    "peak": peaks[peak_key], "unit": "TFLOP/s", "frac": ach / peaks[peak_key],
+                    "peak_source": f"{peaks_src} {peak_key}",
+                    "frac_of_burst": ach / peaks["bf16_tflops"],
+                    "flops_per_launch": fl_launch, "ms_per_launch": dom_ms,
+                    "traffic": traffic_for(dom, args.workload)}
+        else:
+            # fp32 runs on the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flop
+            # (FMA) x 1.965 GHz (max SM clock) = 74.4 TFLOP/s
+            alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+            roof = {"bound": "alu", "kernel": dom, "achieved": ach, "peak": alu_peak,
+                    "unit": "TFLOP/s", "frac": ach / alu_peak,
+                    "peak_source": "derived: 148 SMs x 128 FP32 FMA/clk x 1.965 GHz",
+                    "flops_per_launch": fl_launch, "ms_per_launch": dom_ms, "traffic": None}
 
     e2e = None
     if not args.no_e2e:

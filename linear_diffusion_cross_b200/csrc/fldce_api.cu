@@ -464,7 +464,10 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
     if (p == nullptr) return FLDCE_ERR_INVALID_ARG;
     p->cfg = *cfg;
     p->elt = cfg->dtype == FLDCE_BF16 ? 2 : 4;
-    p->Vpad = (int64_t)round_up((size_t)cfg->V, 8);
+    // G rows start on 128-byte boundaries so every TMA box row of G is one
+    // whole cache line (a 16-byte-aligned but ragged stride costs an extra
+    // sector per box row in both gradient GEMMs).
+    p->Vpad = (int64_t)round_up((size_t)cfg->V, cfg->dtype == FLDCE_BF16 ? 64 : 32);
     p->tile_v = cfg->dtype == FLDCE_BF16 ? kBN : kSimtTile;
     p->n_vt = cdiv(cfg->V, p->tile_v);
     int64_t chunk = cfg->chunk_N;
