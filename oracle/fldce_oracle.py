@@ -27,6 +27,9 @@ p_n, logit scale s, label smoothing eps, normaliser T and upstream gradient g:
     G[n, v]   = g s (softmax[n, v] - eps/V - (1 - eps) [v = y_n]) / (p_n T)
     dH        = G W,   dW = G^T H,   loss = sum_n loss[n]
 
+With the page's optional bias b, the logits are z = s * (<H[n], W[v]> + b[v])
+and db = sum_n G[n, :].
+
 Readings of points the page leaves open or gets inconsistent (each is also
 listed with its justification in the design notes of the repository):
 
@@ -58,7 +61,7 @@ import numpy as np
 __all__ = [
     "valid_tokens", "resolve_total", "logits", "logsumexp_rows", "partial_lse",
     "merge_partial_lse", "smoothed_ce", "token_coef", "grad_logits", "fldce",
-    "fldce_rows", "fldce_dw_rows", "contract_gradients", "OracleResult",
+    "fldce_rows", "fldce_dw_rows", "contract_gradients", "bias_gradient", "OracleResult",
 ]
 
 
@@ -89,10 +92,14 @@ def resolve_total(total: float, valid: np.ndarray) -> float:
     return float(np.count_nonzero(valid))
 
 
-def logits(H: np.ndarray, W: np.ndarray, logit_scale: float) -> np.ndarray:
-    """z = s * H W^T in float64 (F.linear of the chunk loop, then the scale
-    applied in logsumexp_fwd_kernel and cross_entropy_kernel step 5)."""
-    return logit_scale * (np.asarray(H, np.float64) @ np.asarray(W, np.float64).T)
+def logits(H: np.ndarray, W: np.ndarray, logit_scale: float, bias=None) -> np.ndarray:
+    """z = s * (H W^T + b) in float64 (F.linear(c_x, weight, bias) of the
+    chunk loop, then the scale applied in logsumexp_fwd_kernel and
+    cross_entropy_kernel step 5)."""
+    z = np.asarray(H, np.float64) @ np.asarray(W, np.float64).T
+    if bias is not None:
+        z = z + np.asarray(bias, np.float64)[None, :]
+    return logit_scale * z
 
 
 def logsumexp_rows(z: np.ndarray) -> np.ndarray:
@@ -180,6 +187,11 @@ def contract_gradients(G: np.ndarray, H: np.ndarray, W: np.ndarray):
     return G @ W, G.T @ H
 
 
+def bias_gradient(G: np.ndarray) -> np.ndarray:
+    """db = sum_n G[n, :] (db += c_logits.sum(0) in the chunk loop)."""
+    return G.sum(axis=0)
+
+
 @dataclass
 class OracleResult:
     loss: float
@@ -192,6 +204,7 @@ class OracleResult:
     total: float
     n_valid: int
     n_err: int
+    db: Optional[np.ndarray] = None   # [V] when a bias was given
 
 
 def _top2_gap(z: np.ndarray) -> np.ndarray:
@@ -203,7 +216,7 @@ def _top2_gap(z: np.ndarray) -> np.ndarray:
 
 def fldce(H, W, target, p_mask, *, logit_scale: float = 1.0,
           label_smoothing: float = 0.0, ignore_index: int = -100,
-          total: float = 0.0, grad_out: float = 1.0) -> OracleResult:
+          total: float = 0.0, grad_out: float = 1.0, bias=None) -> OracleResult:
     """The whole method on one batch (fused_linear_cross_entropy_forward with
     the backward scaling), materialising the [N, V] logits in float64.
 
@@ -215,7 +228,7 @@ def fldce(H, W, target, p_mask, *, logit_scale: float = 1.0,
     N, V = H.shape[0], W.shape[0]
     valid, n_err = valid_tokens(y, V, ignore_index)
     T = resolve_total(total, valid)
-    z = logits(H, W, logit_scale)
+    z = logits(H, W, logit_scale, bias)
     lse = logsumexp_rows(z)
     ce = smoothed_ce(z, lse, y, label_smoothing)
     coef = token_coef(valid, p_mask, T)
@@ -225,12 +238,13 @@ def fldce(H, W, target, p_mask, *, logit_scale: float = 1.0,
     return OracleResult(
         loss=float(loss_tok.sum()), loss_per_token=loss_tok, lse=lse,
         argmax=np.argmax(z, axis=1).astype(np.int64), top2_gap=_top2_gap(z),
-        dH=dH, dW=dW, total=T, n_valid=int(valid.sum()), n_err=n_err)
+        dH=dH, dW=dW, total=T, n_valid=int(valid.sum()), n_err=n_err,
+        db=None if bias is None else bias_gradient(G))
 
 
 def fldce_rows(H, W, target, p_mask, rows, *, total: float, logit_scale: float = 1.0,
                label_smoothing: float = 0.0, ignore_index: int = -100,
-               grad_out: float = 1.0, row_block: int = 64) -> OracleResult:
+               grad_out: float = 1.0, row_block: int = 64, bias=None) -> OracleResult:
     """Per-token outputs (lse, loss_n, argmax, dH row) for selected token rows.
 
     Each token's row depends only on its own logits, so any row can be
@@ -247,7 +261,7 @@ def fldce_rows(H, W, target, p_mask, rows, *, total: float, logit_scale: float =
         r = rows[a:a + row_block]
         y = y_all[r]
         valid, _ = valid_tokens(y, V, ignore_index)
-        z = logits(H[r], W, logit_scale)
+        z = logits(H[r], W, logit_scale, bias)
         lse = logsumexp_rows(z)
         ce = smoothed_ce(z, lse, y, label_smoothing)
         coef = token_coef(valid, np.asarray(p_mask)[r], total)
@@ -269,7 +283,7 @@ def fldce_rows(H, W, target, p_mask, rows, *, total: float, logit_scale: float =
 def fldce_dw_rows(H, W, target, p_mask, vocab_rows, *, total: float,
                   logit_scale: float = 1.0, label_smoothing: float = 0.0,
                   ignore_index: int = -100, grad_out: float = 1.0,
-                  row_block: int = 128):
+                  row_block: int = 128, bias=None):
     """dW rows for selected vocabulary entries, and lse / loss of every token.
 
     dW[v] = sum_n G[n, v] H[n] needs every token's lse, so all logits are
@@ -288,7 +302,7 @@ def fldce_dw_rows(H, W, target, p_mask, vocab_rows, *, total: float,
         sl = slice(a, min(N, a + row_block))
         y = y_all[sl]
         valid, _ = valid_tokens(y, V, ignore_index)
-        z = logits(H[sl], W, logit_scale)
+        z = logits(H[sl], W, logit_scale, bias)
         lse = logsumexp_rows(z)
         ce = smoothed_ce(z, lse, y, label_smoothing)
         coef = token_coef(valid, np.asarray(p_mask)[sl], total)

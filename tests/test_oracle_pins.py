@@ -286,7 +286,43 @@ def pin_sampled_variants():
     assert np.allclose(lt, r.loss_per_token, rtol=1e-13, atol=0)
 
 
-PINS = [pin_all_zero_logits, pin_label_smoothing_closed_form, pin_ignored_tokens,
+def pin_bias_autograd_and_fd():
+    """Bias: PyTorch float64 autograd of g * sum CE(s F.linear(H, W, b))/(p T)
+    gives dH, dW and db; central differences in b agree."""
+    H, W, y, p = _case(seed=13, ignore_frac=0.3)
+    rng = np.random.default_rng(5)
+    b = rng.standard_normal(W.shape[0])
+    eps, s_, T, g = 0.15, 0.8, 9.0, 1.3
+    r = O.fldce(H, W, y, p, logit_scale=s_, label_smoothing=eps, total=T, grad_out=g, bias=b)
+    Ht = torch.tensor(H, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    yt = torch.from_numpy(y)
+    ce = F.cross_entropy(s_ * F.linear(Ht, Wt, bt), yt, ignore_index=-100,
+                         label_smoothing=eps, reduction="none")
+    w = torch.where(yt != -100, 1.0 / (torch.from_numpy(p) * T), torch.zeros(len(y), dtype=torch.float64))
+    L = (ce * w).sum()
+    L.backward(torch.tensor(g, dtype=torch.float64))
+    assert abs(r.loss - L.item()) <= 1e-12 * abs(L.item())
+    assert np.allclose(r.dH, Ht.grad.numpy(), rtol=1e-10, atol=1e-14)
+    assert np.allclose(r.dW, Wt.grad.numpy(), rtol=1e-10, atol=1e-14)
+    assert np.allclose(r.db, bt.grad.numpy(), rtol=1e-10, atol=1e-14)
+    h = 1e-6
+    for v in (0, 7, W.shape[0] - 1):
+        bp, bm = b.copy(), b.copy()
+        bp[v] += h
+        bm[v] -= h
+        kw = dict(logit_scale=s_, label_smoothing=eps, total=T)
+        fd = g * (O.fldce(H, W, y, p, bias=bp, **kw).loss - O.fldce(H, W, y, p, bias=bm, **kw).loss) / (2 * h)
+        assert abs(fd - r.db[v]) <= 1e-6 * max(1.0, abs(r.db[v]))
+    # zero bias changes nothing
+    r0 = O.fldce(H, W, y, p, logit_scale=s_, label_smoothing=eps, total=T, grad_out=g,
+                 bias=np.zeros(W.shape[0]))
+    r1 = O.fldce(H, W, y, p, logit_scale=s_, label_smoothing=eps, total=T, grad_out=g)
+    assert np.allclose(r0.dW, r1.dW, rtol=1e-14, atol=0) and abs(r0.loss - r1.loss) <= 1e-14 * abs(r1.loss)
+
+
+PINS = [pin_bias_autograd_and_fd, pin_all_zero_logits, pin_label_smoothing_closed_form, pin_ignored_tokens,
         pin_plain_ce_matches_torch, pin_diffusion_weighting_autograd,
         pin_finite_differences, pin_brute_force_loops, pin_split_merge,
         pin_row_sum_invariant, pin_identical_vocab_rows, pin_permutation_equivariance,
@@ -344,9 +380,11 @@ MUTANTS = {
     "lse_no_max_shift_merge": ("merge_partial_lse", lambda: (
         lambda m, l: np.log(l.sum(axis=1)) + m.max(axis=1))),
     "logits_scale_squared": ("logits", lambda: (
-        lambda H, W, s: s * s * (np.asarray(H, float) @ np.asarray(W, float).T))),
+        lambda H, W, s, bias=None: s * s * (np.asarray(H, float) @ np.asarray(W, float).T
+                                            + (0.0 if bias is None else bias)))),
     "logits_transposed_weight": ("logits", lambda: (
-        lambda H, W, s: s * (np.asarray(H, float) @ np.asarray(W, float)[::-1].T))),
+        lambda H, W, s, bias=None: s * (np.asarray(H, float) @ np.asarray(W, float)[::-1].T
+                                        + (0.0 if bias is None else bias)))),
     "total_counts_ignored": ("resolve_total", lambda: (
         lambda total, valid: float(total) if total > 0 else float(valid.shape[0]))),
     "valid_ignores_range": ("valid_tokens", lambda: (
@@ -355,6 +393,12 @@ MUTANTS = {
         lambda G, H, W: (G @ W, G.T @ np.roll(H, 1, axis=0)))),
     "dH_from_reversed_vocab": ("contract_gradients", lambda: (
         lambda G, H, W: (G @ W[::-1], G.T @ H))),
+    "bias_ignored_in_logits": ("logits", lambda: (
+        lambda H, W, s, bias=None: s * (np.asarray(H, float) @ np.asarray(W, float).T))),
+    "bias_outside_scale": ("logits", lambda: (
+        lambda H, W, s, bias=None: s * (np.asarray(H, float) @ np.asarray(W, float).T)
+        + (0.0 if bias is None else np.asarray(bias, float)[None, :]))),
+    "db_mean_not_sum": ("bias_gradient", lambda: (lambda G: G.mean(axis=0))),
     "lse_off_by_log": ("logsumexp_rows", lambda: (
         lambda z: z.max(axis=1) + np.log(np.exp(z - z.max(axis=1)[:, None]).sum(axis=1) + 1.0))),
 }
