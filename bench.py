@@ -230,22 +230,25 @@ def main():
     H, W = wl.H.to(dev), wl.W.to(dev)
     y, p = wl.target.to(dev), wl.p_mask.to(dev)
     total = wl.total if wl.total > 0 else 0.0
-    if world > 1:
-        # one mean over the whole job's tokens: every rank normalises by the
-        # job-wide count (all ranks hold the same batch here)
-        total = world * (wl.total if wl.total > 0 else wl.n_valid())
+    if world > 1 and total > 0:
+        # an explicit normaliser is the job-wide one (every rank holds a batch
+        # of the workload); a count normaliser is summed across ranks on the
+        # device by the data-parallel step
+        total = world * total
     out = plan.outputs(N, want_argmax=False)
     stream = torch.cuda.current_stream(dev)
 
     dist = None
     if world > 1:
         import torch.distributed as dist
+        from linear_diffusion_cross_b200.dp import LibraryKernels, fwd_bwd_data_parallel
+        kern = LibraryKernels(plan)
 
     def step():
-        plan.fwd_bwd(H, W, y, p, total, 1.0, out=out, stream=stream)
-        if dist is not None:
-            dist.all_reduce(out["dW"])
-            dist.all_reduce(out["loss"])
+        if dist is None:
+            plan.fwd_bwd(H, W, y, p, total, 1.0, out=out, stream=stream)
+        else:
+            fwd_bwd_data_parallel(kern, H, W, y, p, total=total, out=out)
 
     def barrier():
         if dist is not None:
@@ -400,10 +403,13 @@ def measure_e2e(plan, wl, total, args, dev, stream, dist):
         dW_.copy_(hW, non_blocking=True)
         dy.copy_(hy, non_blocking=True)
         dp.copy_(hp, non_blocking=True)
-        plan.fwd_bwd(dH_, dW_, dy, dp, total, 1.0, out=out, stream=stream)
-        if dist is not None:
-            dist.all_reduce(out["dW"])
-            dist.all_reduce(out["loss"])
+        if dist is None:
+            plan.fwd_bwd(dH_, dW_, dy, dp, total, 1.0, out=out, stream=stream)
+        else:
+            from linear_diffusion_cross_b200.dp import LibraryKernels, fwd_bwd_data_parallel
+            if not hasattr(measure_e2e, "_kern"):
+                measure_e2e._kern = LibraryKernels(plan)
+            fwd_bwd_data_parallel(measure_e2e._kern, dH_, dW_, dy, dp, total=total, out=out)
         hloss.copy_(out["loss"], non_blocking=True)
 
     for _ in range(2):

@@ -181,6 +181,69 @@ int fldce_fwd_bwd_noalloc(fldce_handle h,
                           void* dH, void* dW, int32_t* err_count, void* stream);
 
 /*
+ * Extended call: every argument of fldce_fwd_bwd in one struct, plus the
+ * page's optional bias and a device-side normaliser for data-parallel use.
+ * Zero-initialise the struct and set what is needed; fields mean what the
+ * same-named arguments of fldce_fwd_bwd mean, and:
+ *   bias      [device, in, may be NULL] [V] dtype: z = s (<H[n], W[v]> + b[v])
+ *             (the page's F.linear(x, weight, bias) before the scale).
+ *   db        [device, out] [V] dtype (fp32 with FLDCE_FLAG_DW_FP32);
+ *             required when bias is set: db[v] = sum_n G[n, v] (the page's
+ *             db += dlogits.sum(0)), summed in a fixed order.
+ *   count_dev [device, in, may be NULL] 1 int32: when total <= 0, the
+ *             normaliser is *count_dev instead of this call's own count --
+ *             e.g. the job-wide count of valid tokens, summed over
+ *             data-parallel ranks from fldce_count_valid (no host sync).
+ *   dw_ready_event [may be NULL] a cudaEvent_t.  When set, the last token
+ *             chunk computes dW (and db) before dH, and the event is
+ *             recorded on `stream` as soon as dW and db hold their final
+ *             values, so a caller can start reducing dW across ranks on
+ *             another stream while dH is still being computed.
+ */
+typedef struct {
+    const void* H;
+    const void* W;
+    const void* bias;
+    const int64_t* target;
+    const float* p_mask;
+    int64_t N;
+    float total;
+    float grad_out;
+    const int32_t* count_dev;
+    float* loss;
+    float* loss_per_token;
+    float* lse;
+    int32_t* argmax;
+    void* dH;
+    void* dW;
+    void* db;
+    void* workspace;
+    size_t workspace_bytes;
+    int32_t* err_count;
+    void* stream;
+    void* dw_ready_event;
+} fldce_call;
+
+/* fldce_fwd_bwd_ex -- fldce_fwd_bwd with the fields of `call`.
+ * Errors: those of fldce_fwd_bwd (INVALID_ARG also for bias without db). */
+int fldce_fwd_bwd_ex(fldce_handle h, const fldce_call* call);
+
+/* fldce_forward_ex -- fldce_forward with the fields of `call` (dH, dW and db
+ * are not used). */
+int fldce_forward_ex(fldce_handle h, const fldce_call* call);
+
+/*
+ * fldce_count_valid -- *count = number of targets that carry a loss (not
+ * ignore_index and inside [0, V)), written on `stream` into device memory.
+ * The page's target.ne(ignore_index).sum(), without the host round trip; a
+ * data-parallel caller sums it over ranks and passes it as count_dev.
+ *   target [device, in] [N] int64;  count [device, out] 1 int32.
+ * Errors: INVALID_ARG, DEVICE, CUDA.
+ */
+int fldce_count_valid(fldce_handle h, const int64_t* target, int64_t N, int32_t* count,
+                      void* stream);
+
+/*
  * fldce_forward -- the loss sweep alone, for evaluation: loss, and
  * optionally loss_per_token / lse / argmax, with no gradients (the page's
  * logsumexp_fwd plus cross_entropy_kernel step 4, without steps 5-6).
@@ -206,11 +269,25 @@ int fldce_forward(fldce_handle h,
  * event before it and the event after it on the same stream.
  * Errors: INVALID_ARG (null handle, max_calls <= 0), CUDA.
  */
-#define FLDCE_PROF_KINDS 8
+#define FLDCE_PROF_KINDS 9
 int fldce_profile_begin(fldce_handle h, int max_calls);
 int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches);
 /* Name of kernel kind k ("lse_sweep", "g_sweep", "dh_gemm", ...), or NULL. */
 const char* fldce_profile_kind_name(int kind);
+
+/*
+ * fldce_scale -- x[i] *= *g for i < n, in place, on `stream`; the kernel
+ * returns without touching x when *g == 1 (the page's
+ * fused_linear_cross_entropy_backward / elementwise_mul_kernel: scale the
+ * saved gradients by the upstream gradient `do`, skipped when do == 1,
+ * decided on the device instead of by a host round trip).
+ *   x      [device, in/out] n elements of `dtype` (FLDCE_BF16 or FLDCE_FP32),
+ *          16-byte aligned.
+ *   g      [device, in] 1 fp32.
+ * Errors: INVALID_ARG (null pointers with n > 0, n < 0), UNSUPPORTED (dtype),
+ * ALIGN, CUDA.
+ */
+int fldce_scale(void* x, int64_t n, int32_t dtype, const float* g, void* stream);
 
 /* fldce_destroy -- free the plan's host memory (and profiling events).
  * NULL is accepted. */

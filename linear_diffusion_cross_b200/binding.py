@@ -33,10 +33,11 @@ FLDCE_FLAG_DW_FP32 = 0x1
 
 # every symbol include/fldce.h declares
 EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
-           "fldce_fwd_bwd_noalloc", "fldce_forward",
+           "fldce_fwd_bwd_noalloc", "fldce_forward", "fldce_fwd_bwd_ex", "fldce_forward_ex",
+           "fldce_count_valid",
            "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
-           "fldce_destroy", "fldce_strerror", "fldce_version")
-FLDCE_PROF_KINDS = 8
+           "fldce_scale", "fldce_destroy", "fldce_strerror", "fldce_version")
+FLDCE_PROF_KINDS = 9
 
 
 class FldceError(RuntimeError):
@@ -56,6 +57,32 @@ class fldce_config(ctypes.Structure):
         ("logit_scale", ctypes.c_float),
         ("label_smoothing", ctypes.c_float),
         ("ignore_index", ctypes.c_int64),
+    ]
+
+
+class fldce_call(ctypes.Structure):
+    _fields_ = [
+        ("H", ctypes.c_void_p),
+        ("W", ctypes.c_void_p),
+        ("bias", ctypes.c_void_p),
+        ("target", ctypes.c_void_p),
+        ("p_mask", ctypes.c_void_p),
+        ("N", ctypes.c_int64),
+        ("total", ctypes.c_float),
+        ("grad_out", ctypes.c_float),
+        ("count_dev", ctypes.c_void_p),
+        ("loss", ctypes.c_void_p),
+        ("loss_per_token", ctypes.c_void_p),
+        ("lse", ctypes.c_void_p),
+        ("argmax", ctypes.c_void_p),
+        ("dH", ctypes.c_void_p),
+        ("dW", ctypes.c_void_p),
+        ("db", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("err_count", ctypes.c_void_p),
+        ("stream", ctypes.c_void_p),
+        ("dw_ready_event", ctypes.c_void_p),
     ]
 
 
@@ -97,6 +124,14 @@ def load() -> ctypes.CDLL:
     lib.fldce_profile_end.restype = ctypes.c_int
     lib.fldce_profile_kind_name.argtypes = [ctypes.c_int]
     lib.fldce_profile_kind_name.restype = ctypes.c_char_p
+    lib.fldce_fwd_bwd_ex.argtypes = [_P, ctypes.POINTER(fldce_call)]
+    lib.fldce_fwd_bwd_ex.restype = ctypes.c_int
+    lib.fldce_forward_ex.argtypes = [_P, ctypes.POINTER(fldce_call)]
+    lib.fldce_forward_ex.restype = ctypes.c_int
+    lib.fldce_count_valid.argtypes = [_P, _P, _I64, _P, _P]
+    lib.fldce_count_valid.restype = ctypes.c_int
+    lib.fldce_scale.argtypes = [_P, _I64, ctypes.c_int32, _P, _P]
+    lib.fldce_scale.restype = ctypes.c_int
     lib.fldce_destroy.argtypes = [_P]
     lib.fldce_destroy.restype = ctypes.c_int
     lib.fldce_strerror.argtypes = [ctypes.c_int]
@@ -205,6 +240,40 @@ def fldce_profile_kind_name(kind: int) -> str:
     return r.decode() if r is not None else None
 
 
+def make_call(**kw) -> fldce_call:
+    """A zero-initialised fldce_call; tensors become device pointers."""
+    c = fldce_call()
+    for k, v in kw.items():
+        if k == "stream":
+            c.stream = _stream(v)
+        elif k == "dw_ready_event":
+            c.dw_ready_event = None if v is None else (
+                v.cuda_event if isinstance(v, torch.cuda.Event) else int(v))
+        elif k in ("N", "total", "grad_out", "workspace_bytes"):
+            setattr(c, k, v)
+        else:
+            setattr(c, k, _ptr(v))
+    return c
+
+
+def fldce_fwd_bwd_ex(h, call: fldce_call) -> int:
+    return _check(load().fldce_fwd_bwd_ex(h, ctypes.byref(call)), "fldce_fwd_bwd_ex")
+
+
+def fldce_forward_ex(h, call: fldce_call) -> int:
+    return _check(load().fldce_forward_ex(h, ctypes.byref(call)), "fldce_forward_ex")
+
+
+def fldce_count_valid(h, target, N, count, stream=None) -> int:
+    return _check(load().fldce_count_valid(h, _ptr(target), int(N), _ptr(count),
+                                           _stream(stream)), "fldce_count_valid")
+
+
+def fldce_scale(x, n, dtype, g, stream=None) -> int:
+    return _check(load().fldce_scale(_ptr(x), int(n), int(dtype), _ptr(g), _stream(stream)),
+                  "fldce_scale")
+
+
 def fldce_destroy(h) -> int:
     return _check(load().fldce_destroy(h), "fldce_destroy")
 
@@ -260,13 +329,28 @@ class Plan:
         return out
 
     def fwd_bwd(self, H, W, target, p_mask, total: float, grad_out: float = 1.0,
-                out: Optional[dict] = None, stream=None, **kw) -> dict:
+                out: Optional[dict] = None, stream=None, bias=None, count_dev=None,
+                dw_ready_event=None, **kw) -> dict:
         N = int(H.shape[0])
         if out is None:
             out = self.outputs(N, **kw)
-        fldce_fwd_bwd(self.handle, H, W, target, p_mask, N, total, grad_out, out["loss"],
-                      out.get("loss_per_token"), out.get("lse"), out.get("argmax"), out["dH"],
-                      out["dW"], self.workspace, self.workspace_bytes, out["err"], stream)
+            if bias is not None:
+                out["db"] = torch.empty(self.V, device=self.device,
+                                        dtype=torch.float32 if self.dw_fp32 else self.dtype)
+        if bias is None and count_dev is None and dw_ready_event is None:
+            fldce_fwd_bwd(self.handle, H, W, target, p_mask, N, total, grad_out, out["loss"],
+                          out.get("loss_per_token"), out.get("lse"), out.get("argmax"),
+                          out["dH"], out["dW"], self.workspace, self.workspace_bytes,
+                          out["err"], stream)
+        else:
+            call = make_call(H=H, W=W, bias=bias, target=target, p_mask=p_mask, N=N,
+                             total=float(total), grad_out=float(grad_out), count_dev=count_dev,
+                             loss=out["loss"], loss_per_token=out.get("loss_per_token"),
+                             lse=out.get("lse"), argmax=out.get("argmax"), dH=out["dH"],
+                             dW=out["dW"], db=out.get("db"), workspace=self.workspace,
+                             workspace_bytes=self.workspace_bytes, err_count=out["err"],
+                             stream=stream, dw_ready_event=dw_ready_event)
+            fldce_fwd_bwd_ex(self.handle, call)
         return out
 
     def forward(self, H, W, target, p_mask, total: float, out: Optional[dict] = None,

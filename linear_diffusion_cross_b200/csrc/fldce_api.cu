@@ -35,6 +35,7 @@ constexpr int kBN = 256;               // vocab tile of the tensor-core sweeps
 constexpr int kStages = 6;
 constexpr size_t kAlign = 256;
 constexpr size_t kGBudget = size_t(1) << 32;   // G buffer per chunk: at most 4 GiB
+constexpr int kColsumSegs = 8;                  // row segments of the db column sums
 
 using CfgKK = GemmCfg<kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
 using CfgKM = GemmCfg<kStages, false, true>;    // dH: G (K-major), W (MN-major)
@@ -133,6 +134,22 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
     return cudaGetLastError();
 }
 
+// db (+)= column sums of the chunk's G, in a fixed order (two passes).
+cudaError_t launch_colsum(const void* G, bool g_bf16, int64_t ldg, int rows, int64_t V,
+                          float* part, float* acc, bool add, cudaStream_t st) {
+    const int nseg = (int)std::min<int64_t>(kColsumSegs, std::max<int64_t>(1, cdiv(rows, 256)));
+    const int seg_rows = (int)cdiv(rows, nseg);
+    const dim3 grid((unsigned)cdiv(cdiv(V, 2), 128), (unsigned)nseg);
+    if (g_bf16)
+        k_colsum_partial<__nv_bfloat16><<<grid, 128, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(G), ldg, rows, V, seg_rows, part);
+    else
+        k_colsum_partial<float><<<grid, 128, 0, st>>>(static_cast<const float*>(G), ldg, rows, V,
+                                                      seg_rows, part);
+    k_colsum_final<<<(unsigned)cdiv(V, 256), 256, 0, st>>>(part, nseg, V, acc, add ? 1 : 0);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, int sms, cudaStream_t st) {
     const int64_t n8 = n / 8;
     if (n8 == 0) return cudaSuccess;
@@ -152,7 +169,7 @@ cudaError_t launch_simt(const float* A, int64_t sam, int64_t sak, const float* B
 
 struct Layout {
     size_t cnt, part_ml, part_sz, part_am, zy, row_lse2, row_gcoef, row_y, loss_tok, G, dh_acc,
-        dw_acc;
+        dw_acc, db_part, db_acc;
     size_t total;
     int64_t C;        // rows per chunk buffer
     int64_t nchunks;
@@ -162,9 +179,9 @@ struct Layout {
 
 enum ProfKind {
     PK_COUNT = 0, PK_LSE = 1, PK_MERGE = 2, PK_G = 3, PK_DH = 4, PK_DW = 5, PK_FINISH = 6,
-    PK_CONVERT = 7, PK_GAP = -1
+    PK_CONVERT = 7, PK_DB = 8, PK_GAP = -1
 };
-static_assert(FLDCE_PROF_KINDS == 8, "kinds");
+static_assert(FLDCE_PROF_KINDS == 9, "kinds");
 
 struct fldce_plan {
     fldce_config cfg;
@@ -220,6 +237,8 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
     L.dh_acc = take(p->cfg.dtype == FLDCE_BF16 ? (size_t)C * p->cfg.D * 4 : 0);
     const bool acc = L.nchunks > 1 && !dw_out_fp32(p);
     L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
+    L.db_part = take((size_t)kColsumSegs * p->cfg.V * 4);
+    L.db_acc = take((size_t)p->cfg.V * 4);
     L.total = off;
     return L;
 }
@@ -233,10 +252,27 @@ int check_device(DeviceInfo* d) {
 }
 
 // The shared body of fldce_fwd_bwd and fldce_forward.
-int run(fldce_handle h, const void* H, const void* W, const int64_t* target, const float* p_mask,
-        int64_t N, float total, float grad_out, float* loss, float* loss_tok_out, float* lse_out,
-        int32_t* argmax_out, void* dH, void* dW, void* workspace, size_t workspace_bytes,
-        int32_t* err_count, void* stream, bool backward) {
+int run(fldce_handle h, const fldce_call& call, bool backward) {
+    const void* H = call.H;
+    const void* W = call.W;
+    const int64_t* target = call.target;
+    const float* p_mask = call.p_mask;
+    const int64_t N = call.N;
+    const float total = call.total, grad_out = call.grad_out;
+    float* loss = call.loss;
+    float* loss_tok_out = call.loss_per_token;
+    float* lse_out = call.lse;
+    int32_t* argmax_out = call.argmax;
+    void* dH = call.dH;
+    void* dW = call.dW;
+    void* workspace = call.workspace;
+    const size_t workspace_bytes = call.workspace_bytes;
+    int32_t* err_count = call.err_count;
+    void* stream = call.stream;
+    const void* bias = call.bias;
+    void* db = call.db;
+    if (backward && bias != nullptr && db == nullptr) return FLDCE_ERR_INVALID_ARG;
+    if (!aligned16(bias) || (backward && !aligned16(db))) return FLDCE_ERR_ALIGN;
     if (h == nullptr || loss == nullptr || N < 0 || N > h->cfg.max_N) return FLDCE_ERR_INVALID_ARG;
     if (N > 0 && (H == nullptr || W == nullptr || target == nullptr)) return FLDCE_ERR_INVALID_ARG;
     if (backward && (dW == nullptr || (N > 0 && dH == nullptr))) return FLDCE_ERR_INVALID_ARG;
@@ -262,6 +298,8 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
     float* row_lse2 = reinterpret_cast<float*>(ws + L.row_lse2);
     float* row_gcoef = reinterpret_cast<float*>(ws + L.row_gcoef);
     int32_t* row_y = reinterpret_cast<int32_t*>(ws + L.row_y);
+    float* db_part = reinterpret_cast<float*>(ws + L.db_part);
+    float* db_acc = reinterpret_cast<float*>(ws + L.db_acc);
     float* loss_tok = loss_tok_out != nullptr ? loss_tok_out
                                               : reinterpret_cast<float*>(ws + L.loss_tok);
     const bool bf16 = cfg.dtype == FLDCE_BF16;
@@ -282,6 +320,8 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         prof_mark(h, PK_COUNT, st);
     } else if (backward) {
         FLDCE_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * D * (dw_out_fp32(h) ? 4 : h->elt), st));
+        if (bias != nullptr)
+            FLDCE_CUDA(cudaMemsetAsync(db, 0, (size_t)V * (dw_out_fp32(h) ? 4 : h->elt), st));
     }
 
     const bool fp32_dw = dw_out_fp32(h);
@@ -309,6 +349,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         lp.part_sz = eps > 0.f ? part_sz : nullptr;
         lp.part_am = argmax_out != nullptr ? part_am : nullptr;
         lp.zy = zy;
+        lp.bias = bf16 ? static_cast<const __nv_bfloat16*>(bias) : nullptr;
 
         CUtensorMap mH_k, mH_mn, mG_k, mG_mn;
         if (bf16) {
@@ -318,7 +359,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
                                                    &cnt->dev_err, dev.sms, st)));
         } else {
             const float* Hc = static_cast<const float*>(H) + r0 * D;
-            SimtLse e{lp};
+            SimtLse e{lp, static_cast<const float*>(bias)};
             FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
                                    e, st));
         }
@@ -341,6 +382,7 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         mp.part_am = argmax_out != nullptr ? part_am : nullptr;
         mp.zy = zy;
         mp.cnt = cnt;
+        mp.count_dev = call.count_dev;
         mp.loss_tok = loss_tok + r0;
         mp.lse_out = lse_out != nullptr ? lse_out + r0 : nullptr;
         mp.am_out = argmax_out != nullptr ? argmax_out + r0 : nullptr;
@@ -355,6 +397,16 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
         // dW: one chunk writes the output directly; several chunks store, then
         // reduce-add, fp32 partial sums (into dW itself when it is fp32).
         const int simt_mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : 2);
+        const bool dw_first = call.dw_ready_event != nullptr && ci + 1 == L.nchunks;
+        // db is final once the last chunk's column sums are in: cast it out
+        auto finish_db = [&]() -> int {
+            if (bias == nullptr || ci + 1 != L.nchunks) return FLDCE_OK;
+            k_cast_out<<<(unsigned)cdiv(V, 256), 256, 0, st>>>(db_acc, db, V,
+                                                              dw_out_fp32(h) ? 0 : 1);
+            FLDCE_CUDA(cudaGetLastError());
+            prof_mark(h, PK_DB, st);
+            return FLDCE_OK;
+        };
         if (bf16) {
             __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(ws + L.G);
             GEpi::Params gp;
@@ -367,9 +419,15 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             gp.ycol = row_y;
             gp.eps_over_V = eps / (float)V;
             gp.one_minus_eps = 1.f - eps;
+            gp.bias = static_cast<const __nv_bfloat16*>(bias);
             FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, 1, gp, &cnt->dev_err,
                                                  dev.sms, st)));
             prof_mark(h, PK_G, st);
+            if (bias != nullptr) {
+                FLDCE_CUDA(launch_colsum(G, true, h->Vpad, rows, V, db_part, db_acc, ci > 0, st));
+                prof_mark(h, PK_DB, st);
+                if (int e = finish_db()) return e;
+            }
             if (!make_map(&mG_k, G, V, rows, h->Vpad, 64, 128)) return FLDCE_ERR_CUDA;
             if (!make_map(&mG_mn, G, V, rows, h->Vpad, 64, 64)) return FLDCE_ERR_CUDA;
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
@@ -379,63 +437,94 @@ int run(fldce_handle h, const void* H, const void* W, const int64_t* target, con
             // idle in its last round, the vocabulary is split in two halves
             // whose fp32 partials are reduce-added into a zeroed buffer (two
             // addends: the sum does not depend on their order).
-            const int pairs = std::max(1, dev.sms / 2);
-            const int64_t dh_tiles = cdiv(rows, CfgKM::PAIR_M) * cdiv(D, CfgKM::BN);
-            const bool dh_split = cdiv(V, CfgKM::BK) >= 8 &&
-                                  wave_efficiency(2 * dh_tiles, pairs) >
-                                      wave_efficiency(dh_tiles, pairs) + 0.03;
-            StoreEpi::Params hp;
-            float* dh_acc = reinterpret_cast<float*>(ws + L.dh_acc);
-            void* dHc = static_cast<__nv_bfloat16*>(dH) + r0 * D;
-            if (dh_split) {
-                FLDCE_CUDA(cudaMemsetAsync(dh_acc, 0, (size_t)rows * D * 4, st));
-                if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
-                hp.mode = WS_ADD;
+            auto do_dh = [&]() -> int {
+                const int pairs = std::max(1, dev.sms / 2);
+                const int64_t dh_tiles = cdiv(rows, CfgKM::PAIR_M) * cdiv(D, CfgKM::BN);
+                const bool dh_split = cdiv(V, CfgKM::BK) >= 8 &&
+                                      wave_efficiency(2 * dh_tiles, pairs) >
+                                          wave_efficiency(dh_tiles, pairs) + 0.03;
+                StoreEpi::Params hp;
+                float* dh_acc = reinterpret_cast<float*>(ws + L.dh_acc);
+                void* dHc = static_cast<__nv_bfloat16*>(dH) + r0 * D;
+                if (dh_split) {
+                    FLDCE_CUDA(cudaMemsetAsync(dh_acc, 0, (size_t)rows * D * 4, st));
+                    if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
+                    hp.mode = WS_ADD;
+                } else {
+                    if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
+                    hp.mode = OUT_BF16;
+                }
+                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1,
+                                                         dh_split ? 2 : 1, hp, &cnt->dev_err,
+                                                         dev.sms, st)));
+                prof_mark(h, PK_DH, st);
+                if (dh_split) {
+                    FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
+                    prof_mark(h, PK_CONVERT, st);
+                }
+                return FLDCE_OK;
+            };
+            // dW = G^T H (K = tokens of the chunk): one chunk writes dW
+            // directly; several store, then reduce-add, fp32 partial sums.
+            auto do_dw = [&]() -> int {
+                StoreEpi::Params wp;
+                if (L.nchunks == 1 && !fp32_dw) {
+                    if (!make_store_map(&wp.omap, dW, D, V, D, 2)) return FLDCE_ERR_CUDA;
+                    wp.mode = OUT_BF16;
+                } else {
+                    if (!make_store_map(&wp.omap, dw_ws, D, V, D, 4)) return FLDCE_ERR_CUDA;
+                    wp.mode = ci == 0 ? WS_STORE : WS_ADD;
+                }
+                FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, 1, wp,
+                                                         &cnt->dev_err, dev.sms, st)));
+                prof_mark(h, PK_DW, st);
+                if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {
+                    FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, dev.sms, st));
+                    prof_mark(h, PK_CONVERT, st);
+                }
+                return FLDCE_OK;
+            };
+            if (dw_first) {
+                if (int e = do_dw()) return e;
+                FLDCE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(call.dw_ready_event), st));
+                if (int e = do_dh()) return e;
             } else {
-                if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
-                hp.mode = OUT_BF16;
-            }
-            FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1,
-                                                     dh_split ? 2 : 1, hp, &cnt->dev_err,
-                                                     dev.sms, st)));
-            prof_mark(h, PK_DH, st);
-            if (dh_split) {
-                FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
-                prof_mark(h, PK_CONVERT, st);
-            }
-
-            StoreEpi::Params wp;
-            if (L.nchunks == 1 && !fp32_dw) {
-                if (!make_store_map(&wp.omap, dW, D, V, D, 2)) return FLDCE_ERR_CUDA;
-                wp.mode = OUT_BF16;
-            } else {
-                if (!make_store_map(&wp.omap, dw_ws, D, V, D, 4)) return FLDCE_ERR_CUDA;
-                wp.mode = ci == 0 ? WS_STORE : WS_ADD;
-            }
-            FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, 1, wp,
-                                                     &cnt->dev_err, dev.sms, st)));
-            prof_mark(h, PK_DW, st);
-            if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {
-                FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, dev.sms, st));
-                prof_mark(h, PK_CONVERT, st);
+                if (int e = do_dh()) return e;
+                if (int e = do_dw()) return e;
             }
         } else {
             float* G = reinterpret_cast<float*>(ws + L.G);
             const float* Hc = static_cast<const float*>(H) + r0 * D;
-            SimtG ge{c, V, h->Vpad, rows, row_lse2, row_gcoef, row_y, eps / (float)V, 1.f - eps, G};
+            SimtG ge{c,     V,         h->Vpad,          rows,
+                     row_lse2, row_gcoef, row_y,   eps / (float)V, 1.f - eps, G,
+                     static_cast<const float*>(bias)};
             FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
                                    ge, st));
             prof_mark(h, PK_G, st);
+            if (bias != nullptr) {
+                FLDCE_CUDA(launch_colsum(G, false, h->Vpad, rows, V, db_part, db_acc, ci > 0, st));
+                prof_mark(h, PK_DB, st);
+                if (int e = finish_db()) return e;
+            }
             SimtStore hs{rows, D, D, static_cast<float*>(dH) + r0 * D, nullptr, 0};
+            SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, simt_mode};
+            if (dw_first) {
+                FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
+                prof_mark(h, PK_DW, st);
+                FLDCE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(call.dw_ready_event), st));
+            }
             FLDCE_CUDA(launch_simt(G, h->Vpad, 1, static_cast<const float*>(W), 1, D, rows, D,
                                    (int)V, hs, st));
             prof_mark(h, PK_DH, st);
-            SimtStore wsd{(int)V, D, D, static_cast<float*>(dW), dw_ws, simt_mode};
-            FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
-            prof_mark(h, PK_DW, st);
+            if (!dw_first) {
+                FLDCE_CUDA(launch_simt(G, 1, h->Vpad, Hc, 1, D, (int)V, D, rows, wsd, st));
+                prof_mark(h, PK_DW, st);
+            }
         }
     }
 
+    if (backward && N == 0 && call.dw_ready_event != nullptr)
+        FLDCE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(call.dw_ready_event), st));
     k_finish<<<1, 1024, 0, st>>>(loss_tok, N, cnt, loss, err_count);
     FLDCE_CUDA(cudaGetLastError());
     prof_mark(h, PK_FINISH, st);
@@ -497,8 +586,57 @@ int fldce_fwd_bwd(fldce_handle h, const void* H, const void* W, const int64_t* t
                   const float* p_mask, int64_t N, float total, float grad_out, float* loss,
                   float* loss_per_token, float* lse, int32_t* argmax, void* dH, void* dW,
                   void* workspace, size_t workspace_bytes, int32_t* err_count, void* stream) {
-    return run(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse, argmax, dH,
-               dW, workspace, workspace_bytes, err_count, stream, true);
+    fldce_call c{};
+    c.H = H;
+    c.W = W;
+    c.target = target;
+    c.p_mask = p_mask;
+    c.N = N;
+    c.total = total;
+    c.grad_out = grad_out;
+    c.loss = loss;
+    c.loss_per_token = loss_per_token;
+    c.lse = lse;
+    c.argmax = argmax;
+    c.dH = dH;
+    c.dW = dW;
+    c.workspace = workspace;
+    c.workspace_bytes = workspace_bytes;
+    c.err_count = err_count;
+    c.stream = stream;
+    return run(h, c, true);
+}
+
+int fldce_fwd_bwd_ex(fldce_handle h, const fldce_call* call) {
+    if (call == nullptr) return FLDCE_ERR_INVALID_ARG;
+    return run(h, *call, true);
+}
+
+int fldce_forward_ex(fldce_handle h, const fldce_call* call) {
+    if (call == nullptr) return FLDCE_ERR_INVALID_ARG;
+    fldce_call c = *call;
+    c.dH = nullptr;
+    c.dW = nullptr;
+    c.db = nullptr;
+    c.grad_out = 1.f;
+    return run(h, c, false);
+}
+
+int fldce_count_valid(fldce_handle h, const int64_t* target, int64_t N, int32_t* count,
+                      void* stream) {
+    if (h == nullptr || count == nullptr || N < 0 || (N > 0 && target == nullptr))
+        return FLDCE_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int s = check_device(&dev)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(count, 0, sizeof(int32_t), st) != cudaSuccess) return FLDCE_ERR_CUDA;
+    if (N > 0) {
+        const int blocks = (int)std::min<int64_t>(cdiv(N, 256), 4 * (int64_t)dev.sms);
+        k_count_valid_only<<<blocks, 256, 0, st>>>(target, N, h->cfg.V, h->cfg.ignore_index,
+                                                   count);
+        if (cudaGetLastError() != cudaSuccess) return FLDCE_ERR_CUDA;
+    }
+    return FLDCE_OK;
 }
 
 }  // extern "C"
@@ -539,22 +677,54 @@ int fldce_fwd_bwd_noalloc(fldce_handle h, const void* H, const void* W, const in
     if (int s = check_device(&dev)) return s;
     void* scratch = nullptr;
     if (int s = static_scratch(&scratch)) return s;
-    return run(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse, argmax, dH,
-               dW, scratch, FLDCE_STATIC_SCRATCH_BYTES, err_count, stream, true);
+    return fldce_fwd_bwd(h, H, W, target, p_mask, N, total, grad_out, loss, loss_per_token, lse,
+                         argmax, dH, dW, scratch, FLDCE_STATIC_SCRATCH_BYTES, err_count, stream);
 }
 
 int fldce_forward(fldce_handle h, const void* H, const void* W, const int64_t* target,
                   const float* p_mask, int64_t N, float total, float* loss, float* loss_per_token,
                   float* lse, int32_t* argmax, void* workspace, size_t workspace_bytes,
                   int32_t* err_count, void* stream) {
-    return run(h, H, W, target, p_mask, N, total, 1.f, loss, loss_per_token, lse, argmax, nullptr,
-               nullptr, workspace, workspace_bytes, err_count, stream, false);
+    fldce_call c{};
+    c.H = H;
+    c.W = W;
+    c.target = target;
+    c.p_mask = p_mask;
+    c.N = N;
+    c.total = total;
+    c.grad_out = 1.f;
+    c.loss = loss;
+    c.loss_per_token = loss_per_token;
+    c.lse = lse;
+    c.argmax = argmax;
+    c.workspace = workspace;
+    c.workspace_bytes = workspace_bytes;
+    c.err_count = err_count;
+    c.stream = stream;
+    return run(h, c, false);
+}
+
+int fldce_scale(void* x, int64_t n, int32_t dtype, const float* g, void* stream) {
+    if (n < 0) return FLDCE_ERR_INVALID_ARG;
+    if (n == 0) return FLDCE_OK;
+    if (x == nullptr || g == nullptr) return FLDCE_ERR_INVALID_ARG;
+    if (dtype != FLDCE_BF16 && dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
+    if (!aligned16(x)) return FLDCE_ERR_ALIGN;
+    DeviceInfo dev;
+    if (int s = check_device(&dev)) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(cdiv(n / 8, 256), 8 * (int64_t)dev.sms));
+    if (dtype == FLDCE_BF16)
+        k_scale<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(x), n, g);
+    else
+        k_scale<float><<<blocks, 256, 0, st>>>(static_cast<float*>(x), n, g);
+    return cudaGetLastError() == cudaSuccess ? FLDCE_OK : FLDCE_ERR_CUDA;
 }
 
 int fldce_profile_begin(fldce_handle h, int max_calls) {
     if (h == nullptr || max_calls <= 0) return FLDCE_ERR_INVALID_ARG;
     const int64_t chunks = cdiv(h->cfg.max_N, h->chunk);
-    const size_t need = (size_t)max_calls * (size_t)(4 + 6 * chunks);
+    const size_t need = (size_t)max_calls * (size_t)(5 + 7 * chunks);
     while (h->ev.size() < need) {
         cudaEvent_t e;
         if (cudaEventCreate(&e) != cudaSuccess) return FLDCE_ERR_CUDA;
@@ -592,7 +762,7 @@ int fldce_profile_end(fldce_handle h, double* ms, int32_t* launches) {
 const char* fldce_profile_kind_name(int kind) {
     static const char* names[FLDCE_PROF_KINDS] = {"count_targets", "lse_sweep", "merge",
                                                   "g_sweep", "dh_gemm", "dw_gemm", "finish",
-                                                  "convert"};
+                                                  "convert", "db_colsum"};
     return (kind >= 0 && kind < FLDCE_PROF_KINDS) ? names[kind] : nullptr;
 }
 

@@ -26,6 +26,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The 32 bias values of columns [c0, c0 + 32) (0 past V), added to the raw
+// accumulator before the logit scale: z = s (<H, W_v> + b_v), as the page's
+// F.linear(x, weight, bias) followed by the scale.
+__device__ __forceinline__ void load_bias32(const __nv_bfloat16* bias, int64_t c0, int64_t V,
+                                            float (&b)[32]) {
+    if (c0 + 32 <= V) {
+        const uint4* q = reinterpret_cast<const uint4*>(bias + c0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint4 w = __ldg(q + k);
+            const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+                b[8 * k + 2 * e] = f.x;
+                b[8 * k + 2 * e + 1] = f.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) b[i] = (c0 + i < V) ? __bfloat162float(bias[c0 + i]) : 0.f;
+    }
+}
+
 // Walk the eight 32-column chunks of this thread's accumulator row with the
 // next chunk's TMEM load in flight while the current one is processed;
 // `f(r, j)` sees chunk j.  The accumulator is released to the MMA warp as
@@ -64,6 +88,7 @@ struct LseEpi {
         float* part_sz;          // [n_vt][ld_part] sum of acc, or null
         int32_t* part_am;        // [n_vt][ld_part] argmax column, or null
         float* zy;               // [ld_part] target logit z[n, y_n]
+        const __nv_bfloat16* bias;   // [V] or null
     };
 
     template <class Cfg>
@@ -82,7 +107,17 @@ struct LseEpi {
         const bool want_am = p.part_am != nullptr, want_sz = p.part_sz != nullptr;
         float mx = -CUDART_INF_F, l = 0.f, sz = 0.f, zyv = 0.f, amv = -CUDART_INF_F;
         int am = 0;
-        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
+        for_each_chunk(acc, [&](const uint32_t (&rin)[32], int j) {
+            uint32_t r[32];
+            if (p.bias != nullptr) {
+                float b[32];
+                load_bias32(p.bias, n0 + 32 * j, p.V, b);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(rin[i]) + b[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = rin[i];
+            }
             float tv[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) tv[i] = __uint_as_float(r[i]) * p.c;
@@ -182,6 +217,7 @@ struct GEpi {
         const int32_t* ycol;     // [chunk] validated target or -1
         float eps_over_V;
         float one_minus_eps;
+        const __nv_bfloat16* bias;   // [V] or null
     };
 
     template <class Cfg>
@@ -204,7 +240,17 @@ struct GEpi {
         const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
         for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
             float g[32];
-            if (gc != 0.f) {
+            if (p.bias != nullptr) {
+                float b[32];
+                load_bias32(p.bias, n0 + 32 * j, p.V, b);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    g[i] = fmaf(gc, ex2(fmaf(__uint_as_float(r[i]) + b[i], p.c, -L2)), -base);
+                if (gc == 0.f) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) g[i] = 0.f;
+                }
+            } else if (gc != 0.f) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     g[i] = fmaf(gc, ex2(fmaf(__uint_as_float(r[i]), p.c, -L2)), -base);
@@ -301,6 +347,20 @@ __global__ void k_count_targets(const int64_t* __restrict__ target, int64_t N, i
     }
 }
 
+// The valid count alone, for fldce_count_valid (count zeroed by the caller).
+__global__ void k_count_valid_only(const int64_t* __restrict__ target, int64_t N, int64_t V,
+                                   int64_t ignore_index, int32_t* count) {
+    int valid = 0;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t y = target[i];
+        if (y != ignore_index && y >= 0 && y < V) ++valid;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) valid += __shfl_xor_sync(0xffffffffu, valid, o);
+    if ((threadIdx.x & 31) == 0 && valid) atomicAdd(count, valid);
+}
+
 struct MergeParams {
     int rows;                 // tokens in this chunk
     int ld_part;              // partial row stride
@@ -315,6 +375,7 @@ struct MergeParams {
     const int32_t* part_am;   // null when argmax is not wanted
     const float* zy;
     const Counters* cnt;
+    const int32_t* count_dev; // job-wide valid count supplied by the caller, or null
     float* loss_tok;          // chunk's per-token loss
     float* lse_out;           // chunk's lse output or null
     int32_t* am_out;          // chunk's argmax output or null
@@ -347,7 +408,8 @@ __global__ void k_merge_rows(MergeParams p) {
     const bool valid = (y != p.ignore_index) && y >= 0 && y < p.V;
     float loss = 0.f, gcoef = 0.f;
     if (valid) {
-        const float T = p.total > 0.f ? p.total : (float)p.cnt->n_valid;
+        const float T = p.total > 0.f ? p.total
+                        : (float)(p.count_dev != nullptr ? *p.count_dev : p.cnt->n_valid);
         const float pm = p.p_mask != nullptr ? p.p_mask[m] : 1.f;
         const float coef = 1.f / (pm * T);
         float ce = lse - p.zy[m];
@@ -409,6 +471,88 @@ __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __re
     }
 }
 
+// x *= *g in place, 8 elements per thread and step; nothing to do when *g == 1.
+template <class T>
+__global__ void k_scale(T* __restrict__ x, int64_t n, const float* __restrict__ g) {
+    const float gv = *g;
+    if (gv == 1.f) return;
+    const int64_t n8 = n / 8;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if constexpr (sizeof(T) == 2) {
+            uint4 w = reinterpret_cast<uint4*>(x)[i];
+            uint32_t* u = &w.x;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u[k]);
+                const float2 f = __bfloat1622float2(v);
+                u[k] = pack_bf16x2(f.x * gv, f.y * gv);
+            }
+            reinterpret_cast<uint4*>(x)[i] = w;
+        } else {
+            float4 a = reinterpret_cast<float4*>(x)[2 * i];
+            float4 b = reinterpret_cast<float4*>(x)[2 * i + 1];
+            a.x *= gv; a.y *= gv; a.z *= gv; a.w *= gv;
+            b.x *= gv; b.y *= gv; b.z *= gv; b.w *= gv;
+            reinterpret_cast<float4*>(x)[2 * i] = a;
+            reinterpret_cast<float4*>(x)[2 * i + 1] = b;
+        }
+    }
+    // the tail (n % 8 elements), one thread
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int64_t i = n8 * 8; i < n; ++i) {
+            if constexpr (sizeof(T) == 2) {
+                x[i] = __float2bfloat16_rn(__bfloat162float(x[i]) * gv);
+            } else {
+                x[i] = x[i] * gv;
+            }
+        }
+    }
+}
+
+// db: column sums of G (the page's db += dlogits.sum(0)) in a fixed order.
+// Pass 1: each thread sums two adjacent columns over one segment of rows.
+template <class T>
+__global__ void k_colsum_partial(const T* __restrict__ G, int64_t ldg, int rows, int64_t V,
+                                 int seg_rows, float* __restrict__ part) {
+    const int64_t v = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (v >= V) return;
+    const int r0 = blockIdx.y * seg_rows;
+    const int r1 = min(rows, r0 + seg_rows);
+    float a0 = 0.f, a1 = 0.f;
+    for (int r = r0; r < r1; ++r) {
+        const T* row = G + (size_t)r * ldg + v;
+        if constexpr (sizeof(T) == 2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(row));
+            a0 += f.x;
+            a1 += f.y;
+        } else {
+            a0 += row[0];
+            a1 += row[1];
+        }
+    }
+    part[(size_t)blockIdx.y * V + v] = a0;
+    if (v + 1 < V) part[(size_t)blockIdx.y * V + v + 1] = a1;
+}
+
+// Pass 2: db_acc[v] (=, or +=) sum of the segment partials, in segment order.
+__global__ void k_colsum_final(const float* __restrict__ part, int nseg, int64_t V,
+                               float* __restrict__ acc, int add) {
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= V) return;
+    float s = 0.f;
+    for (int k = 0; k < nseg; ++k) s += part[(size_t)k * V + v];
+    acc[v] = add ? acc[v] + s : s;
+}
+
+// fp32 -> bf16 or fp32 copy, one element per thread (short vectors, any n).
+__global__ void k_cast_out(const float* __restrict__ src, void* dst, int64_t n, int to_bf16) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    if (to_bf16) static_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(src[i]);
+    else static_cast<float*>(dst)[i] = src[i];
+}
+
 // ======================================================================
 // fp32 CUDA-core path: a 64x64-tile SIMT GEMM whose tile is staged in shared
 // memory and handed to an epilogue.  Used for the fp32 element type, where
@@ -418,12 +562,15 @@ constexpr int kSimtTile = 64;
 
 struct SimtLse {
     LseEpi::Params p;
+    const float* bias;        // [V] fp32 or null
     __device__ void operator()(float (*C)[kSimtTile + 1], int m0, int64_t n0, int nt) const {
         const int r = threadIdx.x;
         if (r >= kSimtTile) return;
         const int m = m0 + r;
         if (m >= p.rows) return;
         const int ncols = (int)((p.V - n0) < kSimtTile ? (p.V - n0) : kSimtTile);
+        if (bias != nullptr)
+            for (int i = 0; i < ncols; ++i) C[r][i] += bias[n0 + i];
         float mx = -CUDART_INF_F, sz = 0.f;
         int am = 0;
         for (int i = 0; i < ncols; ++i) {
@@ -451,6 +598,7 @@ struct SimtG {
     const int32_t* ycol;
     float eps_over_V, one_minus_eps;
     float* G;
+    const float* bias;        // [V] fp32 or null
     __device__ void operator()(float (*C)[kSimtTile + 1], int m0, int64_t n0, int) const {
         for (int idx = threadIdx.x; idx < kSimtTile * kSimtTile; idx += blockDim.x) {
             const int r = idx / kSimtTile, i = idx % kSimtTile;
@@ -460,7 +608,8 @@ struct SimtG {
             const float gc = gcoef[m];
             float g = 0.f;
             if (gc != 0.f && v < V) {
-                g = gc * exp2f(C[r][i] * c - lse2[m]) - gc * eps_over_V;
+                const float a = C[r][i] + (bias != nullptr ? bias[v] : 0.f);
+                g = gc * exp2f(a * c - lse2[m]) - gc * eps_over_V;
                 if (v == ycol[m]) g -= gc * one_minus_eps;
             }
             G[(size_t)m * ldg + v] = g;

@@ -1,0 +1,77 @@
+"""Data-parallel fwd+bwd over token shards (torch.distributed, NCCL on GPUs).
+
+The page's sequence-parallel style (``LinearLossParallel``) shards the tokens
+(x and target) across ranks and replicates the weight and bias.  The loss and
+the weight gradients are sums over tokens, so the one exchange step is a sum
+over ranks:
+
+1. the normaliser: with ``total <= 0`` (the page's 'mean' over non-ignored
+   targets) each rank counts its valid targets on the device
+   (``fldce_count_valid``) and the counts are summed across ranks, so every
+   rank divides by the job-wide count with no host round trip;
+2. each rank runs the fused call on its own tokens with that count;
+   its dH rows are final (they depend only on its tokens);
+3. dW, db and the loss are summed across ranks.  The library records an
+   event as soon as dW (and db) are final -- it computes the last chunk's dW
+   before its dH for this -- so their reduction runs on a side stream while
+   dH is still being computed.
+
+Every rank issues the same collectives in the same order.  ``LibraryKernels``
+binds the per-rank steps to libfldce; the steps are an argument so the
+exchange logic can be exercised with another implementation (the CPU tests
+run it on gloo ranks).
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+import torch.distributed as dist
+
+from . import binding as B
+
+
+class LibraryKernels:
+    """The per-rank steps, on the GPU through the C ABI."""
+
+    def __init__(self, plan: B.Plan):
+        self.plan = plan
+        self._event = torch.cuda.Event()
+        self._side = torch.cuda.Stream(device=plan.device)
+
+    def count_valid(self, target: torch.Tensor) -> torch.Tensor:
+        count = torch.empty(1, dtype=torch.int32, device=self.plan.device)
+        B.fldce_count_valid(self.plan.handle, target, target.shape[0], count)
+        return count
+
+    def fwd_bwd(self, H, W, target, p_mask, total, grad_out, count, bias, out):
+        return self.plan.fwd_bwd(H, W, target, p_mask, total, grad_out, out=out, bias=bias,
+                                 count_dev=count, dw_ready_event=self._event)
+
+    def reduce_weight_grads(self, tensors, group):
+        """Sum dW (and db) over ranks on a side stream once they are final."""
+        side = self._side
+        side.wait_event(self._event)
+        with torch.cuda.stream(side):
+            for t in tensors:
+                dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+        torch.cuda.current_stream(self.plan.device).wait_stream(side)
+        for t in tensors:
+            t.record_stream(side)
+
+
+def fwd_bwd_data_parallel(kernels, H, W, target, p_mask, *, total: float = 0.0,
+                          grad_out: float = 1.0, bias=None, out: Optional[dict] = None,
+                          group=None) -> dict:
+    """One data-parallel step.  H, target, p_mask: this rank's tokens; W, bias:
+    replicated.  ``total > 0`` must already be the job-wide normaliser.
+    Returns this rank's outputs with dW, db and loss summed over ranks."""
+    count = None
+    if total <= 0:
+        count = kernels.count_valid(target)
+        dist.all_reduce(count, op=dist.ReduceOp.SUM, group=group)
+    out = kernels.fwd_bwd(H, W, target, p_mask, total, grad_out, count, bias, out)
+    grads = [out["dW"]] + ([out["db"]] if bias is not None else [])
+    kernels.reduce_weight_grads(grads, group)
+    dist.all_reduce(out["loss"], op=dist.ReduceOp.SUM, group=group)
+    return out

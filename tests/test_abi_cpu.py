@@ -113,7 +113,7 @@ def test_workspace_and_chunking(lib):
 def test_profile_kinds(lib):
     names = [B.fldce_profile_kind_name(k) for k in range(B.FLDCE_PROF_KINDS)]
     assert names == ["count_targets", "lse_sweep", "merge", "g_sweep", "dh_gemm", "dw_gemm",
-                     "finish", "convert"]
+                     "finish", "convert", "db_colsum"]
     assert B.fldce_profile_kind_name(B.FLDCE_PROF_KINDS) is None
 
 
