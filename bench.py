@@ -211,6 +211,8 @@ def main():
                     help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-skip", action="store_true",
+                    help="do not time the FLDCE_FLAG_SKIP_IGNORED variant")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -317,6 +319,36 @@ def main():
                     "peak_source": "derived: 148 SMs x 128 FP32 FMA/clk x 1.965 GHz",
                     "flops_per_launch": fl_launch, "ms_per_launch": dom_ms, "traffic": None}
 
+    # The same step with FLDCE_FLAG_SKIP_IGNORED: only the tokens that carry a
+    # loss enter the GEMMs (identical loss, dH, dW).  Reported beside the
+    # dense line, which does the work the method defines for every token.
+    skip = None
+    if world == 1 and not args.no_skip and wl.H.dtype == torch.bfloat16:
+        splan = B.Plan(D, V, N, dtype=wl.H.dtype, chunk_N=wl.chunk_n,
+                       logit_scale=wl.logit_scale, label_smoothing=wl.label_smoothing,
+                       ignore_index=wl.ignore_index, skip_ignored=True, device=dev)
+        sout = splan.outputs(N, want_argmax=False)
+        for _ in range(args.warmup):
+            splan.fwd_bwd(H, W, y, p, total, 1.0, out=sout, stream=stream)
+        torch.cuda.synchronize(dev)
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            splan.fwd_bwd(H, W, y, p, total, 1.0, out=sout, stream=stream)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        sms = s0.elapsed_time(s1) / args.steps
+        nv = wl.n_valid()
+        skip = {"ms_per_step": sms, "tokens_per_s": N / (sms / 1e3),
+                "valid_tokens": nv, "valid_fraction": nv / N,
+                "tflops_useful_6NvalidDV": 6.0 * nv * D * V / (sms / 1e3) / 1e12,
+                "speedup_vs_dense": ms / sms,
+                "loss_matches_dense": bool(torch.allclose(sout["loss"], out["loss"],
+                                                          rtol=1e-5))}
+        splan.close()
+        del sout
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(plan, wl, total, args, dev, stream, dist)
@@ -344,6 +376,7 @@ def main():
             "kernels_ms_per_step": {k: v[0] / args.steps for k, v in kinds.items()},
             "kernel_share": {k: v[0] / total_kernel_ms for k, v in kinds.items()},
             "gpu_launches": launches,
+            "skip_ignored": skip,
             "e2e": e2e, "cpu_baseline": cb, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -56,7 +56,14 @@ extern "C" {
 #define FLDCE_FP32  1   /* CUDA-core fp32 path (small problems, 1e-5 parity)  */
 
 /* Configuration flags. */
-#define FLDCE_FLAG_DW_FP32  0x1u  /* dW is written as fp32 instead of the dtype */
+#define FLDCE_FLAG_DW_FP32       0x1u  /* dW (and db) are written as fp32 instead of the dtype */
+/* Skip the tokens that carry no loss (ignore_index or out of range): the
+ * valid tokens are compacted on the device and only they enter the GEMMs.
+ * loss, loss_per_token, dH, dW and db are what they are without the flag
+ * (a skipped token's loss is 0, its dH row 0, and it adds nothing to dW);
+ * lse is NaN and argmax is -1 for skipped tokens.  The workspace grows by
+ * about 2 N D + 24 N bytes.  bf16 only (UNSUPPORTED with FLDCE_FP32). */
+#define FLDCE_FLAG_SKIP_IGNORED  0x2u
 
 typedef struct fldce_plan* fldce_handle;
 
@@ -288,6 +295,18 @@ const char* fldce_profile_kind_name(int kind);
  * ALIGN, CUDA.
  */
 int fldce_scale(void* x, int64_t n, int32_t dtype, const float* g, void* stream);
+
+/*
+ * fldce_selftest_wait -- exercise the time-out path of the pipeline waits.
+ * Launches one CTA that waits, with the same bounded wait every GEMM
+ * pipeline stage uses, on a shared-memory mbarrier that nothing ever arrives
+ * on; after `limit_ns` of global time the wait gives up and *status is set
+ * to 1 (the device error bit a timed-out pipeline reports in err_count[1]).
+ * The GPU context stays usable.  limit_ns is clamped to [1000, 2e9].
+ *   status [device, out] 1 int32.
+ * Errors: INVALID_ARG (null status), DEVICE, CUDA.
+ */
+int fldce_selftest_wait(int64_t limit_ns, int32_t* status, void* stream);
 
 /* fldce_destroy -- free the plan's host memory (and profiling events).
  * NULL is accepted. */

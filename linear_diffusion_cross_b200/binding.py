@@ -30,13 +30,14 @@ FLDCE_STATIC_SCRATCH_BYTES = 64 << 20
 FLDCE_BF16 = 0
 FLDCE_FP32 = 1
 FLDCE_FLAG_DW_FP32 = 0x1
+FLDCE_FLAG_SKIP_IGNORED = 0x2
 
 # every symbol include/fldce.h declares
 EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
            "fldce_fwd_bwd_noalloc", "fldce_forward", "fldce_fwd_bwd_ex", "fldce_forward_ex",
            "fldce_count_valid",
            "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
-           "fldce_scale", "fldce_destroy", "fldce_strerror", "fldce_version")
+           "fldce_scale", "fldce_selftest_wait", "fldce_destroy", "fldce_strerror", "fldce_version")
 FLDCE_PROF_KINDS = 9
 
 
@@ -130,6 +131,8 @@ def load() -> ctypes.CDLL:
     lib.fldce_forward_ex.restype = ctypes.c_int
     lib.fldce_count_valid.argtypes = [_P, _P, _I64, _P, _P]
     lib.fldce_count_valid.restype = ctypes.c_int
+    lib.fldce_selftest_wait.argtypes = [_I64, _P, _P]
+    lib.fldce_selftest_wait.restype = ctypes.c_int
     lib.fldce_scale.argtypes = [_P, _I64, ctypes.c_int32, _P, _P]
     lib.fldce_scale.restype = ctypes.c_int
     lib.fldce_destroy.argtypes = [_P]
@@ -274,6 +277,11 @@ def fldce_scale(x, n, dtype, g, stream=None) -> int:
                   "fldce_scale")
 
 
+def fldce_selftest_wait(limit_ns: int, status, stream=None) -> int:
+    return _check(load().fldce_selftest_wait(int(limit_ns), _ptr(status), _stream(stream)),
+                  "fldce_selftest_wait")
+
+
 def fldce_destroy(h) -> int:
     return _check(load().fldce_destroy(h), "fldce_destroy")
 
@@ -286,7 +294,8 @@ class Plan:
 
     def __init__(self, D: int, V: int, max_N: int, *, dtype: torch.dtype = torch.bfloat16,
                  chunk_N: int = 0, logit_scale: float = 1.0, label_smoothing: float = 0.0,
-                 ignore_index: int = -100, dw_fp32: bool = False, device=None):
+                 ignore_index: int = -100, dw_fp32: bool = False, skip_ignored: bool = False,
+                 device=None):
         code = FLDCE_BF16 if dtype == torch.bfloat16 else FLDCE_FP32
         if _TORCH_DTYPE[code] != dtype:
             raise TypeError(f"unsupported dtype {dtype}")
@@ -298,7 +307,8 @@ class Plan:
         self.handle, self.workspace_bytes = fldce_create(
             code, D, V, max_N, chunk_N=chunk_N, logit_scale=logit_scale,
             label_smoothing=label_smoothing, ignore_index=ignore_index,
-            flags=FLDCE_FLAG_DW_FP32 if dw_fp32 else 0)
+            flags=(FLDCE_FLAG_DW_FP32 if dw_fp32 else 0) |
+            (FLDCE_FLAG_SKIP_IGNORED if skip_ignored else 0))
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
 
     def close(self):

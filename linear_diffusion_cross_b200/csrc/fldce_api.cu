@@ -113,11 +113,21 @@ double wave_efficiency(int64_t units, int pairs) {
     return rounds == 0 ? 1.0 : (double)units / (double)(rounds * pairs);
 }
 
+struct DynRows {
+    const int32_t* count = nullptr;   // device-side row count, or null
+    int base = 0;
+    int dim = 0;                      // 1: bounds M, 2: bounds K
+};
+
 template <class Cfg, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64_t N, int64_t K,
                         int n_fastest, int k_splits, const typename Epi::Params& ep, int32_t* err,
-                        int sms, cudaStream_t st) {
+                        int sms, cudaStream_t st, DynRows dyn = DynRows()) {
     GemmGeom g;
+    g.dyn_count = dyn.count;
+    g.dyn_base = dyn.base;
+    g.dyn_dim = dyn.count != nullptr ? dyn.dim : 0;
+    g.dyn_cap = dyn.dim == 2 ? (int)K : M;
     g.tiles_m = (int)cdiv(M, Cfg::PAIR_M);
     g.tiles_n = (int)cdiv(N, Cfg::BN);
     g.k_iters = (int)cdiv(K, Cfg::BK);
@@ -136,16 +146,18 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
 
 // db (+)= column sums of the chunk's G, in a fixed order (two passes).
 cudaError_t launch_colsum(const void* G, bool g_bf16, int64_t ldg, int rows, int64_t V,
-                          float* part, float* acc, bool add, cudaStream_t st) {
+                          float* part, float* acc, bool add, cudaStream_t st,
+                          const int32_t* dyn_count = nullptr, int dyn_base = 0) {
     const int nseg = (int)std::min<int64_t>(kColsumSegs, std::max<int64_t>(1, cdiv(rows, 256)));
     const int seg_rows = (int)cdiv(rows, nseg);
     const dim3 grid((unsigned)cdiv(cdiv(V, 2), 128), (unsigned)nseg);
     if (g_bf16)
         k_colsum_partial<__nv_bfloat16><<<grid, 128, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(G), ldg, rows, V, seg_rows, part);
+            static_cast<const __nv_bfloat16*>(G), ldg, rows, V, seg_rows, part, dyn_count,
+            dyn_base);
     else
         k_colsum_partial<float><<<grid, 128, 0, st>>>(static_cast<const float*>(G), ldg, rows, V,
-                                                      seg_rows, part);
+                                                      seg_rows, part, dyn_count, dyn_base);
     k_colsum_final<<<(unsigned)cdiv(V, 256), 256, 0, st>>>(part, nseg, V, acc, add ? 1 : 0);
     return cudaGetLastError();
 }
@@ -170,6 +182,7 @@ cudaError_t launch_simt(const float* A, int64_t sam, int64_t sak, const float* B
 struct Layout {
     size_t cnt, part_ml, part_sz, part_am, zy, row_lse2, row_gcoef, row_y, loss_tok, G, dh_acc,
         dw_acc, db_part, db_acc;
+    size_t c_idx, c_pos, c_H, c_y, c_p, c_loss, c_lse, c_am, c_dH;   // compaction
     size_t total;
     int64_t C;        // rows per chunk buffer
     int64_t nchunks;
@@ -239,6 +252,17 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
     L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
     L.db_part = take((size_t)kColsumSegs * p->cfg.V * 4);
     L.db_acc = take((size_t)p->cfg.V * 4);
+    const bool skip = (p->cfg.flags & FLDCE_FLAG_SKIP_IGNORED) != 0;
+    const size_t n = skip ? (size_t)std::max<int64_t>(N, 1) : 0;
+    L.c_idx = take(n * 4);
+    L.c_pos = take(n * 4);
+    L.c_H = take(n * p->cfg.D * 2);
+    L.c_y = take(n * 8);
+    L.c_p = take(n * 4);
+    L.c_loss = take(n * 4);
+    L.c_lse = take(n * 4);
+    L.c_am = take(n * 4);
+    L.c_dH = take(n * p->cfg.D * 2);
     L.total = off;
     return L;
 }
@@ -303,6 +327,22 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
     float* loss_tok = loss_tok_out != nullptr ? loss_tok_out
                                               : reinterpret_cast<float*>(ws + L.loss_tok);
     const bool bf16 = cfg.dtype == FLDCE_BF16;
+    const bool skip = (cfg.flags & FLDCE_FLAG_SKIP_IGNORED) != 0;
+    // compaction buffers (FLDCE_FLAG_SKIP_IGNORED) and the caller's outputs
+    int32_t* c_idx = reinterpret_cast<int32_t*>(ws + L.c_idx);
+    int32_t* c_pos = reinterpret_cast<int32_t*>(ws + L.c_pos);
+    __nv_bfloat16* c_H = reinterpret_cast<__nv_bfloat16*>(ws + L.c_H);
+    int64_t* c_y = reinterpret_cast<int64_t*>(ws + L.c_y);
+    float* c_p = reinterpret_cast<float*>(ws + L.c_p);
+    float* c_loss = reinterpret_cast<float*>(ws + L.c_loss);
+    float* c_lse = reinterpret_cast<float*>(ws + L.c_lse);
+    int32_t* c_am = reinterpret_cast<int32_t*>(ws + L.c_am);
+    __nv_bfloat16* c_dH = reinterpret_cast<__nv_bfloat16*>(ws + L.c_dH);
+    float* const user_loss_tok = loss_tok_out;
+    float* const user_lse = lse_out;
+    int32_t* const user_am = argmax_out;
+    void* const user_dH = dH;
+    const int32_t* dynp = nullptr;           // device-side row count of the compacted tokens
     const float s = cfg.logit_scale, eps = cfg.label_smoothing;
     const float c = s * 1.4426950408889634f;
 
@@ -318,6 +358,27 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         k_count_targets<<<blocks, 256, 0, st>>>(target, N, V, cfg.ignore_index, cnt);
         FLDCE_CUDA(cudaGetLastError());
         prof_mark(h, PK_COUNT, st);
+        if (skip) {
+            // compact the tokens that carry a loss; everything below runs on
+            // them, with row counts read on the device (no host sync)
+            k_compact_valid<<<1, 1024, 0, st>>>(target, N, V, cfg.ignore_index, c_idx, c_pos,
+                                                &cnt->n_compact);
+            FLDCE_CUDA(cudaGetLastError());
+            const int gb = (int)std::min<int64_t>(cdiv(N * (D / 8), 256), 8 * (int64_t)dev.sms);
+            k_gather_rows<<<gb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(H), target,
+                                              p_mask, c_idx, &cnt->n_compact, N, D, c_H, c_y,
+                                              c_p);
+            FLDCE_CUDA(cudaGetLastError());
+            prof_mark(h, PK_COUNT, st);
+            H = c_H;
+            target = c_y;
+            p_mask = c_p;
+            loss_tok = c_loss;
+            lse_out = user_lse != nullptr ? c_lse : nullptr;
+            argmax_out = user_am != nullptr ? c_am : nullptr;
+            if (backward) dH = c_dH;
+            dynp = &cnt->n_compact;
+        }
     } else if (backward) {
         FLDCE_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * D * (dw_out_fp32(h) ? 4 : h->elt), st));
         if (bias != nullptr)
@@ -326,6 +387,17 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
 
     const bool fp32_dw = dw_out_fp32(h);
     float* dw_ws = fp32_dw ? static_cast<float*>(dW) : reinterpret_cast<float*>(ws + L.dw_acc);
+
+    if (skip && backward && N > 0) {
+        // with no token to carry a loss the dW GEMM has no K rows: zero the
+        // buffer its first chunk would have written
+        const bool direct = L.nchunks == 1 && !fp32_dw;
+        void* dst = direct ? dW : static_cast<void*>(dw_ws);
+        const int64_t b16 = (int64_t)V * D * (direct ? 2 : 4) / 16;
+        k_zero_if_none<<<(unsigned)std::min<int64_t>(cdiv(b16, 256), 8 * (int64_t)dev.sms), 256, 0,
+                         st>>>(dynp, dst, b16);
+        FLDCE_CUDA(cudaGetLastError());
+    }
 
     CUtensorMap mW_k, mW_mn;
     if (bf16 && N > 0) {
@@ -356,7 +428,8 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
             if (!make_map(&mH_k, Hc, D, rows, D, 64, 128)) return FLDCE_ERR_CUDA;
             FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, 1, lp,
-                                                   &cnt->dev_err, dev.sms, st)));
+                                                   &cnt->dev_err, dev.sms, st,
+                                                   DynRows{dynp, (int)r0, 1})));
         } else {
             const float* Hc = static_cast<const float*>(H) + r0 * D;
             SimtLse e{lp, static_cast<const float*>(bias)};
@@ -383,6 +456,8 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         mp.zy = zy;
         mp.cnt = cnt;
         mp.count_dev = call.count_dev;
+        mp.dyn_count = dynp;
+        mp.dyn_base = (int)r0;
         mp.loss_tok = loss_tok + r0;
         mp.lse_out = lse_out != nullptr ? lse_out + r0 : nullptr;
         mp.am_out = argmax_out != nullptr ? argmax_out + r0 : nullptr;
@@ -421,10 +496,11 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
             gp.one_minus_eps = 1.f - eps;
             gp.bias = static_cast<const __nv_bfloat16*>(bias);
             FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, 1, gp, &cnt->dev_err,
-                                                 dev.sms, st)));
+                                                 dev.sms, st, DynRows{dynp, (int)r0, 1})));
             prof_mark(h, PK_G, st);
             if (bias != nullptr) {
-                FLDCE_CUDA(launch_colsum(G, true, h->Vpad, rows, V, db_part, db_acc, ci > 0, st));
+                FLDCE_CUDA(launch_colsum(G, true, h->Vpad, rows, V, db_part, db_acc, ci > 0, st,
+                                         dynp, (int)r0));
                 prof_mark(h, PK_DB, st);
                 if (int e = finish_db()) return e;
             }
@@ -456,7 +532,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
                 }
                 FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1,
                                                          dh_split ? 2 : 1, hp, &cnt->dev_err,
-                                                         dev.sms, st)));
+                                                         dev.sms, st, DynRows{dynp, (int)r0, 1})));
                 prof_mark(h, PK_DH, st);
                 if (dh_split) {
                     FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
@@ -476,7 +552,8 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
                     wp.mode = ci == 0 ? WS_STORE : WS_ADD;
                 }
                 FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, 1, wp,
-                                                         &cnt->dev_err, dev.sms, st)));
+                                                         &cnt->dev_err, dev.sms, st,
+                                                         DynRows{dynp, (int)r0, 2})));
                 prof_mark(h, PK_DW, st);
                 if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {
                     FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, dev.sms, st));
@@ -523,6 +600,14 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         }
     }
 
+    if (skip && N > 0) {
+        const int sb = (int)std::min<int64_t>(cdiv(N * (D / 8), 256), 8 * (int64_t)dev.sms);
+        k_scatter_rows<<<sb, 256, 0, st>>>(c_pos, N, D, c_dH,
+                                           backward ? static_cast<__nv_bfloat16*>(user_dH) : nullptr,
+                                           c_loss, user_loss_tok, c_lse, user_lse, c_am, user_am);
+        FLDCE_CUDA(cudaGetLastError());
+        prof_mark(h, PK_CONVERT, st);
+    }
     if (backward && N == 0 && call.dw_ready_event != nullptr)
         FLDCE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(call.dw_ready_event), st));
     k_finish<<<1, 1024, 0, st>>>(loss_tok, N, cnt, loss, err_count);
@@ -544,7 +629,10 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
         return FLDCE_ERR_INVALID_ARG;
     if (!std::isfinite(cfg->logit_scale) || cfg->logit_scale == 0.f) return FLDCE_ERR_INVALID_ARG;
     if (cfg->dtype != FLDCE_BF16 && cfg->dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
-    if ((cfg->flags & ~FLDCE_FLAG_DW_FP32) != 0) return FLDCE_ERR_UNSUPPORTED;
+    if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED)) != 0)
+        return FLDCE_ERR_UNSUPPORTED;
+    if ((cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0 && cfg->dtype != FLDCE_BF16)
+        return FLDCE_ERR_UNSUPPORTED;
     if (cfg->D % 8 != 0) return FLDCE_ERR_UNSUPPORTED;
     if (cfg->V > (int64_t(1) << 31) - 1 || cfg->max_N > (int64_t(1) << 31) - 1 ||
         cfg->D > (int64_t(1) << 31) - 1)
@@ -718,6 +806,15 @@ int fldce_scale(void* x, int64_t n, int32_t dtype, const float* g, void* stream)
         k_scale<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<__nv_bfloat16*>(x), n, g);
     else
         k_scale<float><<<blocks, 256, 0, st>>>(static_cast<float*>(x), n, g);
+    return cudaGetLastError() == cudaSuccess ? FLDCE_OK : FLDCE_ERR_CUDA;
+}
+
+int fldce_selftest_wait(int64_t limit_ns, int32_t* status, void* stream) {
+    if (status == nullptr) return FLDCE_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if (int s = check_device(&dev)) return s;
+    const uint64_t lim = (uint64_t)std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 2000000000);
+    k_selftest_wait<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(lim, status);
     return cudaGetLastError() == cudaSuccess ? FLDCE_OK : FLDCE_ERR_CUDA;
 }
 

@@ -97,7 +97,7 @@ struct LseEpi {
         const int m = t.row0 + t.row;
         const int64_t n0 = t.col0;
         const int nt = (int)(n0 / Cfg::BN);
-        const bool live = m < p.rows;
+        const bool live = m < (t.rows_dyn >= 0 ? t.rows_dyn : p.rows);
         int yrel = -1;
         if (live) {
             const int64_t y = p.target[m];
@@ -227,7 +227,7 @@ struct GEpi {
         const int64_t n0 = t.col0;
         float gc = 0.f, L2 = 0.f;
         int yrel = -1;
-        if (m < p.rows) {
+        if (m < (t.rows_dyn >= 0 ? t.rows_dyn : p.rows)) {
             gc = p.gcoef[m];
             if (gc != 0.f) {
                 L2 = p.lse2[m];
@@ -321,7 +321,7 @@ struct Counters {
     int32_t n_valid;   // targets != ignore_index and inside [0, V)
     int32_t n_err;     // targets != ignore_index outside [0, V)
     int32_t dev_err;   // FLDCE_DEV_ERR_* bits raised by kernels
-    int32_t pad;
+    int32_t n_compact; // compacted tokens (FLDCE_FLAG_SKIP_IGNORED)
 };
 
 // Count the tokens that carry a loss (the page's target.ne(ignore_index).sum(),
@@ -347,6 +347,114 @@ __global__ void k_count_targets(const int64_t* __restrict__ target, int64_t N, i
     }
 }
 
+// Stable compaction of the tokens that carry a loss (one block): idx lists
+// their positions in increasing order, pos maps a position to its compacted
+// row (or -1), *count = how many.  Skipping the rest changes no result: an
+// ignored token's loss is 0, its dH row is 0 and it adds nothing to dW.
+__global__ void k_compact_valid(const int64_t* __restrict__ target, int64_t N, int64_t V,
+                                int64_t ignore_index, int32_t* __restrict__ idx,
+                                int32_t* __restrict__ pos, int32_t* count) {
+    __shared__ int warp_tot[32];
+    const int T = blockDim.x;
+    const int64_t seg = (N + T - 1) / T;
+    const int64_t a = threadIdx.x * seg;
+    const int64_t b = min(N, a + seg);
+    int c = 0;
+    for (int64_t i = a; i < b; ++i) {
+        const int64_t y = target[i];
+        c += (y != ignore_index && y >= 0 && y < V) ? 1 : 0;
+    }
+    // exclusive scan of c over the block
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = lane < (T >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += t;
+        }
+        warp_tot[lane] = v;    // inclusive totals per warp
+    }
+    __syncthreads();
+    int off = incl - c + (w > 0 ? warp_tot[w - 1] : 0);
+    for (int64_t i = a; i < b; ++i) {
+        const int64_t y = target[i];
+        if (y != ignore_index && y >= 0 && y < V) {
+            idx[off] = (int32_t)i;
+            pos[i] = off++;
+        } else {
+            pos[i] = -1;
+        }
+    }
+    if (threadIdx.x == T - 1) *count = off;
+}
+
+// Gather the compacted rows: Hc[i] = H[idx[i]], yc, pc.  The 256 rows after
+// the count are zero-filled: a chunk's last GEMM tile may read up to 255
+// rows past it, and zeros (not stale workspace bits) keep them out of dW.
+__global__ void k_gather_rows(const __nv_bfloat16* __restrict__ H, const int64_t* __restrict__ y,
+                              const float* __restrict__ p, const int32_t* __restrict__ idx,
+                              const int32_t* count, int64_t N, int64_t D,
+                              __nv_bfloat16* __restrict__ Hc, int64_t* __restrict__ yc,
+                              float* __restrict__ pc) {
+    const int n = *count;
+    const int64_t lim = min(N, (int64_t)n + 256);
+    const int64_t per_row = D / 8;                 // 16-byte vectors per row
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < lim * per_row;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / per_row, c = e - i * per_row;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i < n) v = reinterpret_cast<const uint4*>(H + (int64_t)idx[i] * D)[c];
+        reinterpret_cast<uint4*>(Hc + i * D)[c] = v;
+        if (c == 0) {
+            yc[i] = i < n ? y[idx[i]] : (int64_t)-1;
+            pc[i] = i < n ? (p != nullptr ? p[idx[i]] : 1.f) : 1.f;
+        }
+    }
+}
+
+// Scatter back: dH[i] = dHc[pos[i]] (zero row for skipped tokens), and the
+// per-token outputs (loss 0, lse NaN, argmax -1 for skipped tokens).
+__global__ void k_scatter_rows(const int32_t* __restrict__ pos, int64_t N, int64_t D,
+                               const __nv_bfloat16* __restrict__ dHc, __nv_bfloat16* __restrict__ dH,
+                               const float* __restrict__ loss_c, float* loss_out,
+                               const float* __restrict__ lse_c, float* lse_out,
+                               const int32_t* __restrict__ am_c, int32_t* am_out) {
+    const int64_t per_row = D / 8;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < N * per_row;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / per_row, c = e - i * per_row;
+        const int32_t q = pos[i];
+        if (dH != nullptr) {
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (q >= 0) v = reinterpret_cast<const uint4*>(dHc + (int64_t)q * D)[c];
+            reinterpret_cast<uint4*>(dH + i * D)[c] = v;
+        }
+        if (c == 0) {
+            if (loss_out != nullptr) loss_out[i] = q >= 0 ? loss_c[q] : 0.f;
+            if (lse_out != nullptr) lse_out[i] = q >= 0 ? lse_c[q] : CUDART_NAN_F;
+            if (am_out != nullptr) am_out[i] = q >= 0 ? am_c[q] : -1;
+        }
+    }
+}
+
+// When no token carries a loss, the dW GEMM has no K rows and writes nothing:
+// zero its destination instead (a no-op otherwise).
+__global__ void k_zero_if_none(const int32_t* count, void* dst, int64_t bytes16) {
+    if (*count != 0) return;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < bytes16;
+         i += (int64_t)gridDim.x * blockDim.x)
+        reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+}
+
 // The valid count alone, for fldce_count_valid (count zeroed by the caller).
 __global__ void k_count_valid_only(const int64_t* __restrict__ target, int64_t N, int64_t V,
                                    int64_t ignore_index, int32_t* count) {
@@ -362,7 +470,9 @@ __global__ void k_count_valid_only(const int64_t* __restrict__ target, int64_t N
 }
 
 struct MergeParams {
-    int rows;                 // tokens in this chunk
+    int rows;                 // tokens in this chunk (with dyn_count: the capacity)
+    const int32_t* dyn_count; // compacted-token count, or null
+    int dyn_base;             // first compacted row of this chunk
     int ld_part;              // partial row stride
     int n_vt;                 // vocab tiles
     int64_t V;
@@ -391,6 +501,16 @@ struct MergeParams {
 __global__ void k_merge_rows(MergeParams p) {
     const int m = blockIdx.x * blockDim.x + threadIdx.x;
     if (m >= p.rows) return;
+    if (p.dyn_count != nullptr && m >= *p.dyn_count - p.dyn_base) {
+        // past the compacted tokens: no loss, zero gradient row
+        p.loss_tok[m] = 0.f;
+        if (p.row_lse2 != nullptr) {
+            p.row_lse2[m] = 0.f;
+            p.row_gcoef[m] = 0.f;
+            p.row_y[m] = -1;
+        }
+        return;
+    }
     float M2 = -CUDART_INF_F;
     int kbest = 0;
     for (int k = 0; k < p.n_vt; ++k) {
@@ -471,6 +591,19 @@ __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __re
     }
 }
 
+// One CTA waits, bounded, on an mbarrier that never completes its phase.
+__global__ void k_selftest_wait(uint64_t limit_ns, int32_t* status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const bool done = mbar_wait_bounded(smem_u32(&bar), 0u, limit_ns);
+    __syncthreads();
+    if (threadIdx.x == 0) *status = done ? 0 : FLDCE_DEV_ERR_TIMEOUT;
+}
+
 // x *= *g in place, 8 elements per thread and step; nothing to do when *g == 1.
 template <class T>
 __global__ void k_scale(T* __restrict__ x, int64_t n, const float* __restrict__ g) {
@@ -514,9 +647,11 @@ __global__ void k_scale(T* __restrict__ x, int64_t n, const float* __restrict__ 
 // Pass 1: each thread sums two adjacent columns over one segment of rows.
 template <class T>
 __global__ void k_colsum_partial(const T* __restrict__ G, int64_t ldg, int rows, int64_t V,
-                                 int seg_rows, float* __restrict__ part) {
+                                 int seg_rows, float* __restrict__ part,
+                                 const int32_t* dyn_count, int dyn_base) {
     const int64_t v = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
     if (v >= V) return;
+    if (dyn_count != nullptr) rows = max(0, min(rows, *dyn_count - dyn_base));
     const int r0 = blockIdx.y * seg_rows;
     const int r1 = min(rows, r0 + seg_rows);
     float a0 = 0.f, a1 = 0.f;

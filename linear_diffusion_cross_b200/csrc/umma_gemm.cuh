@@ -73,10 +73,35 @@ struct GemmGeom {
     int k_splits;         // K ranges per tile (1 or 2)
     int num_tiles;        // tiles_m * tiles_n
     int n_fastest;        // 1: consecutive tiles walk n first (share the A panel)
+    // Optional row count known only on the device (compacted tokens): the
+    // live rows are clamp(*dyn_count - dyn_base, 0, dyn_cap), bounding M
+    // (dyn_dim == 1) or K (dyn_dim == 2).  The host sizes the launch for
+    // dyn_cap rows; every CTA reads the same count at start.
+    const int32_t* dyn_count;
+    int dyn_base;
+    int dyn_cap;
+    int dyn_dim;
 };
+
+// Apply the device-side row count of `g` (if any); returns the live rows or -1.
+__device__ __forceinline__ int apply_dyn_rows(GemmGeom& g) {
+    if (g.dyn_dim == 0) return -1;
+    int n = *g.dyn_count - g.dyn_base;
+    n = n < 0 ? 0 : (n > g.dyn_cap ? g.dyn_cap : n);
+    if (g.dyn_dim == 1) {
+        g.tiles_m = (n + 255) / 256;
+        g.num_tiles = g.tiles_m * g.tiles_n;
+    } else {
+        g.k_iters = (n + 63) / 64;
+        if (g.k_iters < 2 * g.k_splits) g.k_splits = 1;
+        if (g.k_iters == 0) g.num_tiles = 0;
+    }
+    return n;
+}
 
 // Where the current tile of this thread sits.
 struct TileCtx {
+    int rows_dyn;         // live rows from the device-side count, or -1
     int row0;             // output row of TMEM lane 0 of this CTA
     int64_t col0;         // first output column of the tile
     int split;            // K split index
@@ -146,9 +171,11 @@ struct Stager {
 template <class Cfg, class Epi>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmGeom geom, const __grid_constant__ typename Epi::Params ep,
+                 const GemmGeom geom_in, const __grid_constant__ typename Epi::Params ep,
                  int32_t* err) {
     constexpr int S = Cfg::STAGES;
+    GemmGeom geom = geom_in;
+    const int rows_dyn = apply_dyn_rows(geom);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -321,8 +348,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 break;
             }
             tc_fence_after();
-            TileCtx t{mt * Cfg::PAIR_M + (int)rank * Cfg::BM, (int64_t)nt * Cfg::BN, split, row,
-                      q, lane};
+            TileCtx t{rows_dyn, mt * Cfg::PAIR_M + (int)rank * Cfg::BM, (int64_t)nt * Cfg::BN,
+                      split, row, q, lane};
             AccRow acc{tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * Cfg::BN),
                        lead_tempty0 + 8u * (uint32_t)b, lane};
             Epi::template run<Cfg>(ep, t, acc, st);

@@ -58,6 +58,7 @@ def test_version(lib):
     (dict(D=60), B.FLDCE_ERR_UNSUPPORTED),
     (dict(dtype=7), B.FLDCE_ERR_UNSUPPORTED),
     (dict(flags=0x10), B.FLDCE_ERR_UNSUPPORTED),
+    (dict(dtype=1, flags=0x2), B.FLDCE_ERR_UNSUPPORTED),
 ])
 def test_create_rejects(lib, kw, code):
     args = dict(dtype=B.FLDCE_BF16, D=64, V=100, max_N=10)

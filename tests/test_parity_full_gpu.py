@@ -79,3 +79,31 @@ def test_full_size(name):
         assert abs(loss - loss_ref) <= LOSS_RTOL * abs(loss_ref), (loss, loss_ref)
         info["loss"] = abs(loss - loss_ref) / abs(loss_ref)
     print(name, info)
+
+
+def test_full_size_headline_skip_ignored():
+    """The headline workload with FLDCE_FLAG_SKIP_IGNORED: same loss, dH rows
+    and dW rows as the oracle; lse NaN and dH zero for every skipped token."""
+    from linear_diffusion_cross_b200 import binding as B
+    wl = synth.make("headline", 0)
+    dev = torch.device("cuda")
+    plan = B.Plan(wl.D, wl.V, wl.N, skip_ignored=True, device=dev)
+    g = plan.fwd_bwd(wl.H.to(dev), wl.W.to(dev), wl.target.to(dev), wl.p_mask.to(dev),
+                     wl.total, want_argmax=True)
+    torch.cuda.synchronize()
+    g = {k: v.cpu() for k, v in g.items()}
+    H, W, y, p = oracle_inputs(wl)
+    valid, _ = O.valid_tokens(y, wl.V, wl.ignore_index)
+    ign = ~valid
+    assert torch.count_nonzero(g["dH"][torch.from_numpy(ign)]) == 0
+    assert torch.isnan(g["lse"][torch.from_numpy(ign)]).all()
+    assert (g["argmax"][torch.from_numpy(ign)] == -1).all()
+    rows = np.nonzero(valid)[0][synth.sample_rows(int(valid.sum()), N_SAMPLE_ROWS, 3).numpy()]
+    ref = O.fldce_rows(H, W, y, p, rows, total=wl.total, **oracle_kw(wl))
+    assert maxabs_err(f64(g["dH"])[rows], ref.dH) <= GRAD_TOL["bf16"]
+    assert maxabs_err(g["loss_per_token"].double().numpy()[rows], ref.loss_per_token) <= 1e-3
+    vr = synth.sample_rows(wl.V, N_SAMPLE_VOCAB, 4, [wl.V - 1]).numpy()
+    dWr, _, lt_all = O.fldce_dw_rows(H, W, y, p, vr, total=wl.total, **oracle_kw(wl))
+    assert maxabs_err(f64(g["dW"])[vr], dWr) <= GRAD_TOL["bf16"]
+    loss_ref = float(lt_all.sum())
+    assert abs(float(g["loss"][0]) - loss_ref) <= LOSS_RTOL * abs(loss_ref)
