@@ -351,7 +351,8 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(plan, wl, total, args, dev, stream, dist)
+        e2e = measure_e2e(plan, wl, total, args, dev, stream, dist,
+                          kern if dist is not None else None)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -415,7 +416,7 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measure_e2e(plan, wl, total, args, dev, stream, dist):
+def measure_e2e(plan, wl, total, args, dev, stream, dist, kern=None):
     """Same step through the public API with host buffers: pinned host inputs
     copied to the device and the loss copied back inside every timed step."""
     hH = wl.H.pin_memory()
@@ -436,13 +437,11 @@ def measure_e2e(plan, wl, total, args, dev, stream, dist):
         dW_.copy_(hW, non_blocking=True)
         dy.copy_(hy, non_blocking=True)
         dp.copy_(hp, non_blocking=True)
-        if dist is None:
+        if kern is None:
             plan.fwd_bwd(dH_, dW_, dy, dp, total, 1.0, out=out, stream=stream)
         else:
-            from linear_diffusion_cross_b200.dp import LibraryKernels, fwd_bwd_data_parallel
-            if not hasattr(measure_e2e, "_kern"):
-                measure_e2e._kern = LibraryKernels(plan)
-            fwd_bwd_data_parallel(measure_e2e._kern, dH_, dW_, dy, dp, total=total, out=out)
+            from linear_diffusion_cross_b200.dp import fwd_bwd_data_parallel
+            fwd_bwd_data_parallel(kern, dH_, dW_, dy, dp, total=total, out=out)
         hloss.copy_(out["loss"], non_blocking=True)
 
     for _ in range(2):

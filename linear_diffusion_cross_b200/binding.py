@@ -250,8 +250,12 @@ def make_call(**kw) -> fldce_call:
         if k == "stream":
             c.stream = _stream(v)
         elif k == "dw_ready_event":
-            c.dw_ready_event = None if v is None else (
+            handle = None if v is None else (
                 v.cuda_event if isinstance(v, torch.cuda.Event) else int(v))
+            if v is not None and not handle:
+                # a torch.cuda.Event has no CUDA event until its first record
+                raise ValueError("dw_ready_event has no CUDA event yet: record it once first")
+            c.dw_ready_event = handle
         elif k in ("N", "total", "grad_out", "workspace_bytes"):
             setattr(c, k, v)
         else:

@@ -36,8 +36,13 @@ class LibraryKernels:
 
     def __init__(self, plan: B.Plan):
         self.plan = plan
-        self._event = torch.cuda.Event()
         self._side = torch.cuda.Stream(device=plan.device)
+        # torch creates the CUDA event on its first record; the library records
+        # it by handle, so create it now (a record on an idle stream is free)
+        self._event = torch.cuda.Event()
+        self._event.record(torch.cuda.current_stream(plan.device))
+        if not self._event.cuda_event:
+            raise RuntimeError("could not create the dW-ready CUDA event")
 
     def count_valid(self, target: torch.Tensor) -> torch.Tensor:
         count = torch.empty(1, dtype=torch.int32, device=self.plan.device)

@@ -36,7 +36,9 @@ def test_dp_step_one_rank(chunk, use_bias, total):
         plan = B.Plan(wl.D, wl.V, wl.N, chunk_N=chunk, label_smoothing=0.1, device=dev)
         args = (wl.H.to(dev), wl.W.to(dev), wl.target.to(dev), wl.p_mask.to(dev))
         bias = b.to(dev) if use_bias else None
-        out = fwd_bwd_data_parallel(LibraryKernels(plan), *args, total=total, bias=bias)
+        kern = LibraryKernels(plan)
+        assert kern._event.cuda_event != 0
+        out = fwd_bwd_data_parallel(kern, *args, total=total, bias=bias)
         torch.cuda.synchronize()
         ref = O.fldce(f64(wl.H), f64(wl.W), wl.target.numpy(), f64(wl.p_mask), total=total,
                       label_smoothing=0.1, bias=f64(b) if use_bias else None)
@@ -51,3 +53,27 @@ def test_dp_step_one_rank(chunk, use_bias, total):
         assert torch.equal(plain["dW"], out["dW"]) and torch.equal(plain["dH"], out["dH"])
     finally:
         dist.destroy_process_group()
+
+
+def test_dw_ready_event_fires_after_dw_is_final():
+    """The library records the event once dW is final: a copy of dW taken on
+    another stream right after the event equals the dW the call returns, even
+    while dH (computed after dW in this mode) is still running."""
+    dev = torch.device("cuda", 0)
+    r = synth.Recipe("ev", 1, 4096, 2048, 32000, torch.bfloat16, 0.02, 1e-3)
+    wl = synth.make(r, 8)
+    plan = B.Plan(wl.D, wl.V, wl.N, device=dev)
+    ev = torch.cuda.Event()
+    ev.record(torch.cuda.current_stream(dev))
+    side = torch.cuda.Stream(device=dev)
+    args = (wl.H.to(dev), wl.W.to(dev), wl.target.to(dev), wl.p_mask.to(dev))
+    out = plan.outputs(wl.N)
+    out["dW"].zero_()
+    plan.fwd_bwd(*args, wl.total, out=out, dw_ready_event=ev)
+    side.wait_event(ev)
+    with torch.cuda.stream(side):
+        snap = out["dW"].clone()
+    torch.cuda.synchronize()
+    assert torch.equal(snap, out["dW"]) and torch.count_nonzero(snap) > 0
+    with pytest.raises(ValueError):
+        B.make_call(dw_ready_event=torch.cuda.Event())
