@@ -64,6 +64,9 @@ extern "C" {
  * lse is NaN and argmax is -1 for skipped tokens.  The workspace grows by
  * about 2 N D + 24 N bytes.  bf16 only (UNSUPPORTED with FLDCE_FP32). */
 #define FLDCE_FLAG_SKIP_IGNORED  0x2u
+/* dH is written as fp32 instead of the dtype (e.g. partial dH summed over
+ * vocabulary shards).  Not with FLDCE_FLAG_SKIP_IGNORED. */
+#define FLDCE_FLAG_DH_FP32       0x4u
 
 typedef struct fldce_plan* fldce_handle;
 
@@ -77,6 +80,12 @@ typedef struct {
     float logit_scale;        /* s (the page's logit_scale), finite and nonzero   */
     float label_smoothing;    /* eps in [0, 1]                                    */
     int64_t ignore_index;     /* the page's ignore_index, usually -100            */
+    /* Vocabulary sharding (0, 0 = not sharded).  With vocab_total > 0 this
+     * plan's W is rows [vocab_start, vocab_start + V) of a vocabulary of
+     * vocab_total entries; targets are global ids; only the fldce_vp_* entry
+     * points accept such a plan. */
+    int64_t vocab_start;
+    int64_t vocab_total;
 } fldce_config;
 
 /*
@@ -238,6 +247,32 @@ int fldce_fwd_bwd_ex(fldce_handle h, const fldce_call* call);
 /* fldce_forward_ex -- fldce_forward with the fields of `call` (dH, dW and db
  * are not used). */
 int fldce_forward_ex(fldce_handle h, const fldce_call* call);
+
+/*
+ * Vocabulary-parallel loss (the tensor-parallel tutorial page, section 4:
+ * each shard computes its own softmax denominators, they are combined across
+ * shards, and every shard then works on its own columns).  A plan made with
+ * vocab_total > 0 covers one shard; every rank holds all N tokens.
+ *
+ * fldce_vp_stats -- sweep 1 over this shard: for each token n, 8 fp32 at
+ *   stats[8 n .. 8 n + 7]: m2 (max of z log2 e over the shard), l (sum of
+ *   2^(z log2 e - m2)), z[n, y_n] if y_n is in the shard else 0, s * sum of
+ *   (H W^T + b) over the shard, the shard argmax as int32 bits (global id),
+ *   3 unused.  Uses call->H, W, bias, target, N, workspace, stream.
+ *   stats [device, out] [N][8] fp32.
+ *
+ * fldce_vp_fwd_bwd -- everything after the exchange: `all_stats` holds the
+ *   n_shards shards' stats ([n_shards][N][8], in vocabulary order: the shard
+ *   with the lowest vocab_start first), gathered from every rank.  They are
+ *   merged in that fixed order into lse, the loss (identical on every rank),
+ *   and G for this shard's columns; then dW and db for this shard, and this
+ *   shard's partial dH = G_shard W_shard, which the caller sums over shards.
+ *   Fields of `call` as for fldce_fwd_bwd_ex (argmax and lse are global).
+ * Errors: those of fldce_fwd_bwd_ex; INVALID_ARG for an unsharded plan.
+ */
+int fldce_vp_stats(fldce_handle h, const fldce_call* call, float* stats);
+int fldce_vp_fwd_bwd(fldce_handle h, const fldce_call* call, const float* all_stats,
+                     int32_t n_shards);
 
 /*
  * fldce_count_valid -- *count = number of targets that carry a loss (not

@@ -31,11 +31,12 @@ FLDCE_BF16 = 0
 FLDCE_FP32 = 1
 FLDCE_FLAG_DW_FP32 = 0x1
 FLDCE_FLAG_SKIP_IGNORED = 0x2
+FLDCE_FLAG_DH_FP32 = 0x4
 
 # every symbol include/fldce.h declares
 EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
            "fldce_fwd_bwd_noalloc", "fldce_forward", "fldce_fwd_bwd_ex", "fldce_forward_ex",
-           "fldce_count_valid",
+           "fldce_count_valid", "fldce_vp_stats", "fldce_vp_fwd_bwd",
            "fldce_profile_begin", "fldce_profile_end", "fldce_profile_kind_name",
            "fldce_scale", "fldce_selftest_wait", "fldce_destroy", "fldce_strerror", "fldce_version")
 FLDCE_PROF_KINDS = 9
@@ -58,6 +59,8 @@ class fldce_config(ctypes.Structure):
         ("logit_scale", ctypes.c_float),
         ("label_smoothing", ctypes.c_float),
         ("ignore_index", ctypes.c_int64),
+        ("vocab_start", ctypes.c_int64),
+        ("vocab_total", ctypes.c_int64),
     ]
 
 
@@ -129,6 +132,10 @@ def load() -> ctypes.CDLL:
     lib.fldce_fwd_bwd_ex.restype = ctypes.c_int
     lib.fldce_forward_ex.argtypes = [_P, ctypes.POINTER(fldce_call)]
     lib.fldce_forward_ex.restype = ctypes.c_int
+    lib.fldce_vp_stats.argtypes = [_P, ctypes.POINTER(fldce_call), _P]
+    lib.fldce_vp_stats.restype = ctypes.c_int
+    lib.fldce_vp_fwd_bwd.argtypes = [_P, ctypes.POINTER(fldce_call), _P, ctypes.c_int32]
+    lib.fldce_vp_fwd_bwd.restype = ctypes.c_int
     lib.fldce_count_valid.argtypes = [_P, _P, _I64, _P, _P]
     lib.fldce_count_valid.restype = ctypes.c_int
     lib.fldce_selftest_wait.argtypes = [_I64, _P, _P]
@@ -177,10 +184,12 @@ def fldce_version() -> int:
 
 def fldce_create(dtype: int, D: int, V: int, max_N: int, *, chunk_N: int = 0,
                  logit_scale: float = 1.0, label_smoothing: float = 0.0,
-                 ignore_index: int = -100, flags: int = 0):
+                 ignore_index: int = -100, flags: int = 0, vocab_start: int = 0,
+                 vocab_total: int = 0):
     """Returns (handle, workspace_bytes for max_N)."""
     cfg = fldce_config(int(dtype), int(flags), int(D), int(V), int(max_N), int(chunk_N),
-                       float(logit_scale), float(label_smoothing), int(ignore_index))
+                       float(logit_scale), float(label_smoothing), int(ignore_index),
+                       int(vocab_start), int(vocab_total))
     h = _P()
     ws = ctypes.c_size_t()
     _check(load().fldce_create(ctypes.byref(h), ctypes.byref(cfg), ctypes.byref(ws)),
@@ -271,6 +280,15 @@ def fldce_forward_ex(h, call: fldce_call) -> int:
     return _check(load().fldce_forward_ex(h, ctypes.byref(call)), "fldce_forward_ex")
 
 
+def fldce_vp_stats(h, call: fldce_call, stats) -> int:
+    return _check(load().fldce_vp_stats(h, ctypes.byref(call), _ptr(stats)), "fldce_vp_stats")
+
+
+def fldce_vp_fwd_bwd(h, call: fldce_call, all_stats, n_shards: int) -> int:
+    return _check(load().fldce_vp_fwd_bwd(h, ctypes.byref(call), _ptr(all_stats), int(n_shards)),
+                  "fldce_vp_fwd_bwd")
+
+
 def fldce_count_valid(h, target, N, count, stream=None) -> int:
     return _check(load().fldce_count_valid(h, _ptr(target), int(N), _ptr(count),
                                            _stream(stream)), "fldce_count_valid")
@@ -299,6 +317,7 @@ class Plan:
     def __init__(self, D: int, V: int, max_N: int, *, dtype: torch.dtype = torch.bfloat16,
                  chunk_N: int = 0, logit_scale: float = 1.0, label_smoothing: float = 0.0,
                  ignore_index: int = -100, dw_fp32: bool = False, skip_ignored: bool = False,
+                 dh_fp32: bool = False, vocab_start: int = 0, vocab_total: int = 0,
                  device=None):
         code = FLDCE_BF16 if dtype == torch.bfloat16 else FLDCE_FP32
         if _TORCH_DTYPE[code] != dtype:
@@ -312,7 +331,10 @@ class Plan:
             code, D, V, max_N, chunk_N=chunk_N, logit_scale=logit_scale,
             label_smoothing=label_smoothing, ignore_index=ignore_index,
             flags=(FLDCE_FLAG_DW_FP32 if dw_fp32 else 0) |
-            (FLDCE_FLAG_SKIP_IGNORED if skip_ignored else 0))
+            (FLDCE_FLAG_SKIP_IGNORED if skip_ignored else 0) |
+            (FLDCE_FLAG_DH_FP32 if dh_fp32 else 0),
+            vocab_start=vocab_start, vocab_total=vocab_total)
+        self.dh_fp32 = bool(dh_fp32)
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
 
     def close(self):
@@ -330,7 +352,8 @@ class Plan:
         dev = self.device
         out = {
             "loss": torch.empty(1, dtype=torch.float32, device=dev),
-            "dH": torch.empty(N, self.D, dtype=self.dtype, device=dev),
+            "dH": torch.empty(N, self.D, dtype=torch.float32 if self.dh_fp32 else self.dtype,
+                              device=dev),
             "dW": torch.empty(self.V, self.D,
                               dtype=torch.float32 if self.dw_fp32 else self.dtype, device=dev),
             "err": torch.empty(2, dtype=torch.int32, device=dev),

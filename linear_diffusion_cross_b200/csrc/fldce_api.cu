@@ -198,6 +198,9 @@ static_assert(FLDCE_PROF_KINDS == 9, "kinds");
 
 struct fldce_plan {
     fldce_config cfg;
+    int64_t v0;       // first vocabulary id of this plan's W (0 unsharded)
+    int64_t Vtot;     // total vocabulary (== V unsharded)
+    bool sharded;
     int64_t chunk;    // tokens per chunk
     int64_t Vpad;     // row stride of G (elements)
     int tile_v;       // vocab tile width of the partial statistics
@@ -276,7 +279,11 @@ int check_device(DeviceInfo* d) {
 }
 
 // The shared body of fldce_fwd_bwd and fldce_forward.
-int run(fldce_handle h, const fldce_call& call, bool backward) {
+// mode: MERGE_LOCAL (the whole vocabulary in this plan), MERGE_EMIT_STATS
+// (a shard's sweep 1 and statistics only), MERGE_GATHERED (a shard's
+// backward from every shard's statistics).
+int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_LOCAL,
+        float* stats_out = nullptr, const float* all_stats = nullptr, int n_shards = 0) {
     const void* H = call.H;
     const void* W = call.W;
     const int64_t* target = call.target;
@@ -296,8 +303,14 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
     const void* bias = call.bias;
     void* db = call.db;
     if (backward && bias != nullptr && db == nullptr) return FLDCE_ERR_INVALID_ARG;
+    if (h != nullptr && h->sharded != (mode != MERGE_LOCAL)) return FLDCE_ERR_INVALID_ARG;
+    if (mode == MERGE_EMIT_STATS && stats_out == nullptr) return FLDCE_ERR_INVALID_ARG;
+    if (mode == MERGE_GATHERED && (all_stats == nullptr || n_shards <= 0))
+        return FLDCE_ERR_INVALID_ARG;
     if (!aligned16(bias) || (backward && !aligned16(db))) return FLDCE_ERR_ALIGN;
-    if (h == nullptr || loss == nullptr || N < 0 || N > h->cfg.max_N) return FLDCE_ERR_INVALID_ARG;
+    if (h == nullptr || (loss == nullptr && mode != MERGE_EMIT_STATS) || N < 0 ||
+        N > h->cfg.max_N)
+        return FLDCE_ERR_INVALID_ARG;
     if (N > 0 && (H == nullptr || W == nullptr || target == nullptr)) return FLDCE_ERR_INVALID_ARG;
     if (backward && (dW == nullptr || (N > 0 && dH == nullptr))) return FLDCE_ERR_INVALID_ARG;
     if (!std::isfinite(total) || !std::isfinite(grad_out)) return FLDCE_ERR_INVALID_ARG;
@@ -355,14 +368,14 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
     prof_mark(h, PK_GAP, st);
     if (N > 0) {
         const int blocks = (int)std::min<int64_t>(cdiv(N, 256), 4 * (int64_t)dev.sms);
-        k_count_targets<<<blocks, 256, 0, st>>>(target, N, V, cfg.ignore_index, cnt);
+        k_count_targets<<<blocks, 256, 0, st>>>(target, N, h->Vtot, cfg.ignore_index, cnt);
         FLDCE_CUDA(cudaGetLastError());
         prof_mark(h, PK_COUNT, st);
         if (skip) {
             // compact the tokens that carry a loss; everything below runs on
             // them, with row counts read on the device (no host sync)
-            k_compact_valid<<<1, 1024, 0, st>>>(target, N, V, cfg.ignore_index, c_idx, c_pos,
-                                                &cnt->n_compact);
+            k_compact_valid<<<1, 1024, 0, st>>>(target, N, h->Vtot, cfg.ignore_index, c_idx,
+                                                c_pos, &cnt->n_compact);
             FLDCE_CUDA(cudaGetLastError());
             const int gb = (int)std::min<int64_t>(cdiv(N * (D / 8), 256), 8 * (int64_t)dev.sms);
             k_gather_rows<<<gb, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(H), target,
@@ -419,26 +432,41 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         lp.target = tgt;
         lp.part_ml = part_ml;
         lp.part_sz = eps > 0.f ? part_sz : nullptr;
-        lp.part_am = argmax_out != nullptr ? part_am : nullptr;
+        const bool want_am = argmax_out != nullptr || mode == MERGE_EMIT_STATS;
+        lp.part_am = want_am ? part_am : nullptr;
         lp.zy = zy;
         lp.bias = bf16 ? static_cast<const __nv_bfloat16*>(bias) : nullptr;
+        lp.v0 = h->v0;
 
         CUtensorMap mH_k, mH_mn, mG_k, mG_mn;
         if (bf16) {
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
             if (!make_map(&mH_k, Hc, D, rows, D, 64, 128)) return FLDCE_ERR_CUDA;
-            FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, 1, lp,
-                                                   &cnt->dev_err, dev.sms, st,
-                                                   DynRows{dynp, (int)r0, 1})));
-        } else {
-            const float* Hc = static_cast<const float*>(H) + r0 * D;
-            SimtLse e{lp, static_cast<const float*>(bias)};
-            FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
-                                   e, st));
         }
-        prof_mark(h, PK_LSE, st);
+        // sweep 1 (not needed when every shard's statistics are given)
+        if (mode != MERGE_GATHERED) {
+            if (bf16) {
+                FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, 1, lp,
+                                                       &cnt->dev_err, dev.sms, st,
+                                                       DynRows{dynp, (int)r0, 1})));
+            } else {
+                const float* Hc = static_cast<const float*>(H) + r0 * D;
+                SimtLse e{lp, static_cast<const float*>(bias)};
+                FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V,
+                                       (int)D, e, st));
+            }
+            prof_mark(h, PK_LSE, st);
+        }
 
         MergeParams mp;
+        mp.mode = mode;
+        mp.v0 = h->v0;
+        mp.Vtot = h->Vtot;
+        mp.stats_out = stats_out;
+        mp.all_stats = all_stats;
+        mp.n_shards = n_shards;
+        mp.stats_N = N;
+        mp.stats_row0 = r0;
         mp.rows = rows;
         mp.ld_part = (int)L.C;
         mp.n_vt = (int)h->n_vt;
@@ -452,7 +480,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         mp.p_mask = p_mask != nullptr ? p_mask + r0 : nullptr;
         mp.part_ml = part_ml;
         mp.part_sz = eps > 0.f ? part_sz : nullptr;
-        mp.part_am = argmax_out != nullptr ? part_am : nullptr;
+        mp.part_am = want_am ? part_am : nullptr;
         mp.zy = zy;
         mp.cnt = cnt;
         mp.count_dev = call.count_dev;
@@ -461,13 +489,13 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
         mp.loss_tok = loss_tok + r0;
         mp.lse_out = lse_out != nullptr ? lse_out + r0 : nullptr;
         mp.am_out = argmax_out != nullptr ? argmax_out + r0 : nullptr;
-        mp.row_lse2 = backward ? row_lse2 : nullptr;
+        mp.row_lse2 = backward && mode != MERGE_EMIT_STATS ? row_lse2 : nullptr;
         mp.row_gcoef = row_gcoef;
         mp.row_y = row_y;
         k_merge_rows<<<(unsigned)cdiv(rows, 128), 128, 0, st>>>(mp);
         FLDCE_CUDA(cudaGetLastError());
         prof_mark(h, PK_MERGE, st);
-        if (!backward) continue;
+        if (!backward || mode == MERGE_EMIT_STATS) continue;
 
         // dW: one chunk writes the output directly; several chunks store, then
         // reduce-add, fp32 partial sums (into dW itself when it is fp32).
@@ -492,7 +520,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
             gp.lse2 = row_lse2;
             gp.gcoef = row_gcoef;
             gp.ycol = row_y;
-            gp.eps_over_V = eps / (float)V;
+            gp.eps_over_V = eps / (float)h->Vtot;
             gp.one_minus_eps = 1.f - eps;
             gp.bias = static_cast<const __nv_bfloat16*>(bias);
             FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, 1, gp, &cnt->dev_err,
@@ -520,12 +548,17 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
                                       wave_efficiency(2 * dh_tiles, pairs) >
                                           wave_efficiency(dh_tiles, pairs) + 0.03;
                 StoreEpi::Params hp;
-                float* dh_acc = reinterpret_cast<float*>(ws + L.dh_acc);
+                const bool dh_fp32 = (cfg.flags & FLDCE_FLAG_DH_FP32) != 0;
+                float* dh_acc = dh_fp32 ? static_cast<float*>(dH) + r0 * D
+                                        : reinterpret_cast<float*>(ws + L.dh_acc);
                 void* dHc = static_cast<__nv_bfloat16*>(dH) + r0 * D;
                 if (dh_split) {
                     FLDCE_CUDA(cudaMemsetAsync(dh_acc, 0, (size_t)rows * D * 4, st));
                     if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
                     hp.mode = WS_ADD;
+                } else if (dh_fp32) {
+                    if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
+                    hp.mode = WS_STORE;
                 } else {
                     if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
                     hp.mode = OUT_BF16;
@@ -534,7 +567,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
                                                          dh_split ? 2 : 1, hp, &cnt->dev_err,
                                                          dev.sms, st, DynRows{dynp, (int)r0, 1})));
                 prof_mark(h, PK_DH, st);
-                if (dh_split) {
+                if (dh_split && !dh_fp32) {
                     FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
                     prof_mark(h, PK_CONVERT, st);
                 }
@@ -573,7 +606,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
             float* G = reinterpret_cast<float*>(ws + L.G);
             const float* Hc = static_cast<const float*>(H) + r0 * D;
             SimtG ge{c,     V,         h->Vpad,          rows,
-                     row_lse2, row_gcoef, row_y,   eps / (float)V, 1.f - eps, G,
+                     row_lse2, row_gcoef, row_y,   eps / (float)h->Vtot, 1.f - eps, G,
                      static_cast<const float*>(bias)};
             FLDCE_CUDA(launch_simt(Hc, D, 1, static_cast<const float*>(W), D, 1, rows, V, (int)D,
                                    ge, st));
@@ -610,6 +643,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward) {
     }
     if (backward && N == 0 && call.dw_ready_event != nullptr)
         FLDCE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(call.dw_ready_event), st));
+    if (mode == MERGE_EMIT_STATS) return FLDCE_OK;
     k_finish<<<1, 1024, 0, st>>>(loss_tok, N, cnt, loss, err_count);
     FLDCE_CUDA(cudaGetLastError());
     prof_mark(h, PK_FINISH, st);
@@ -629,10 +663,17 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
         return FLDCE_ERR_INVALID_ARG;
     if (!std::isfinite(cfg->logit_scale) || cfg->logit_scale == 0.f) return FLDCE_ERR_INVALID_ARG;
     if (cfg->dtype != FLDCE_BF16 && cfg->dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
-    if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED)) != 0)
+    if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED | FLDCE_FLAG_DH_FP32)) != 0)
         return FLDCE_ERR_UNSUPPORTED;
-    if ((cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0 && cfg->dtype != FLDCE_BF16)
+    if ((cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0 &&
+        (cfg->dtype != FLDCE_BF16 || (cfg->flags & FLDCE_FLAG_DH_FP32) != 0))
         return FLDCE_ERR_UNSUPPORTED;
+    if (cfg->vocab_total > 0 && (cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0)
+        return FLDCE_ERR_UNSUPPORTED;
+    if (cfg->vocab_total < 0 || cfg->vocab_start < 0 ||
+        (cfg->vocab_total > 0 && cfg->vocab_start + cfg->V > cfg->vocab_total) ||
+        (cfg->vocab_total == 0 && cfg->vocab_start != 0))
+        return FLDCE_ERR_INVALID_ARG;
     if (cfg->D % 8 != 0) return FLDCE_ERR_UNSUPPORTED;
     if (cfg->V > (int64_t(1) << 31) - 1 || cfg->max_N > (int64_t(1) << 31) - 1 ||
         cfg->D > (int64_t(1) << 31) - 1)
@@ -640,6 +681,9 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
     fldce_plan* p = new (std::nothrow) fldce_plan;
     if (p == nullptr) return FLDCE_ERR_INVALID_ARG;
     p->cfg = *cfg;
+    p->sharded = cfg->vocab_total > 0;
+    p->v0 = cfg->vocab_start;
+    p->Vtot = p->sharded ? cfg->vocab_total : cfg->V;
     p->elt = cfg->dtype == FLDCE_BF16 ? 2 : 4;
     // G rows start on 128-byte boundaries so every TMA box row of G is one
     // whole cache line (a 16-byte-aligned but ragged stride costs an extra
@@ -710,6 +754,17 @@ int fldce_forward_ex(fldce_handle h, const fldce_call* call) {
     return run(h, c, false);
 }
 
+int fldce_vp_stats(fldce_handle h, const fldce_call* call, float* stats) {
+    if (call == nullptr) return FLDCE_ERR_INVALID_ARG;
+    return run(h, *call, false, MERGE_EMIT_STATS, stats);
+}
+
+int fldce_vp_fwd_bwd(fldce_handle h, const fldce_call* call, const float* all_stats,
+                     int32_t n_shards) {
+    if (call == nullptr) return FLDCE_ERR_INVALID_ARG;
+    return run(h, *call, true, MERGE_GATHERED, nullptr, all_stats, n_shards);
+}
+
 int fldce_count_valid(fldce_handle h, const int64_t* target, int64_t N, int32_t* count,
                       void* stream) {
     if (h == nullptr || count == nullptr || N < 0 || (N > 0 && target == nullptr))
@@ -720,7 +775,7 @@ int fldce_count_valid(fldce_handle h, const int64_t* target, int64_t N, int32_t*
     if (cudaMemsetAsync(count, 0, sizeof(int32_t), st) != cudaSuccess) return FLDCE_ERR_CUDA;
     if (N > 0) {
         const int blocks = (int)std::min<int64_t>(cdiv(N, 256), 4 * (int64_t)dev.sms);
-        k_count_valid_only<<<blocks, 256, 0, st>>>(target, N, h->cfg.V, h->cfg.ignore_index,
+        k_count_valid_only<<<blocks, 256, 0, st>>>(target, N, h->Vtot, h->cfg.ignore_index,
                                                    count);
         if (cudaGetLastError() != cudaSuccess) return FLDCE_ERR_CUDA;
     }

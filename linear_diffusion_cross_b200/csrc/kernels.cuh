@@ -89,6 +89,7 @@ struct LseEpi {
         int32_t* part_am;        // [n_vt][ld_part] argmax column, or null
         float* zy;               // [ld_part] target logit z[n, y_n]
         const __nv_bfloat16* bias;   // [V] or null
+        int64_t v0;              // first vocabulary id of this shard (0 unsharded)
     };
 
     template <class Cfg>
@@ -100,7 +101,7 @@ struct LseEpi {
         const bool live = m < (t.rows_dyn >= 0 ? t.rows_dyn : p.rows);
         int yrel = -1;
         if (live) {
-            const int64_t y = p.target[m];
+            const int64_t y = p.target[m] - p.v0;      // shard-local column
             if (y >= n0 && y < n0 + Cfg::BN && y < p.V) yrel = (int)(y - n0);
         }
         const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
@@ -469,7 +470,16 @@ __global__ void k_count_valid_only(const int64_t* __restrict__ target, int64_t N
     if ((threadIdx.x & 31) == 0 && valid) atomicAdd(count, valid);
 }
 
+enum MergeMode { MERGE_LOCAL = 0, MERGE_EMIT_STATS = 1, MERGE_GATHERED = 2 };
+
 struct MergeParams {
+    int mode;                 // MergeMode
+    int64_t v0, Vtot;         // shard offset and total vocabulary (0, V unsharded)
+    float* stats_out;         // MERGE_EMIT_STATS: [.][8] rows for this chunk
+    const float* all_stats;   // MERGE_GATHERED: [n_shards][stats_N][8]
+    int n_shards;
+    int64_t stats_N;          // tokens per shard's stats block
+    int64_t stats_row0;       // first token of this chunk
     int rows;                 // tokens in this chunk (with dyn_count: the capacity)
     const int32_t* dyn_count; // compacted-token count, or null
     int dyn_base;             // first compacted row of this chunk
@@ -511,44 +521,76 @@ __global__ void k_merge_rows(MergeParams p) {
         }
         return;
     }
-    float M2 = -CUDART_INF_F;
-    int kbest = 0;
-    for (int k = 0; k < p.n_vt; ++k) {
-        const float v = p.part_ml[(size_t)k * p.ld_part + m].x;
-        if (v > M2) { M2 = v; kbest = k; }
-    }
-    float L = 0.f;
-    for (int k = 0; k < p.n_vt; ++k) {
-        const float2 ml = p.part_ml[(size_t)k * p.ld_part + m];
-        L += ml.y * exp2f(ml.x - M2);
+    const int64_t gm = p.stats_row0 + m;          // token index within the call
+    const int64_t y = p.target[m];
+    const bool valid = (y != p.ignore_index) && y >= 0 && y < p.Vtot;
+    const bool local_y = valid && y - p.v0 >= 0 && y - p.v0 < p.V;
+    float M2 = -CUDART_INF_F, L = 0.f, zyv = 0.f, szv = 0.f;
+    int32_t am = -1;
+    if (p.mode != MERGE_GATHERED) {
+        // this shard's vocab tiles
+        int kbest = 0;
+        for (int k = 0; k < p.n_vt; ++k) {
+            const float v = p.part_ml[(size_t)k * p.ld_part + m].x;
+            if (v > M2) { M2 = v; kbest = k; }
+        }
+        for (int k = 0; k < p.n_vt; ++k) {
+            const float2 ml = p.part_ml[(size_t)k * p.ld_part + m];
+            L += ml.y * exp2f(ml.x - M2);
+        }
+        if (local_y) zyv = p.zy[m];
+        if (p.part_sz != nullptr) {
+            float sz = 0.f;
+            for (int k = 0; k < p.n_vt; ++k) sz += p.part_sz[(size_t)k * p.ld_part + m];
+            szv = p.s * sz;
+        }
+        if (p.part_am != nullptr) am = p.part_am[(size_t)kbest * p.ld_part + m] + (int32_t)p.v0;
+        if (p.mode == MERGE_EMIT_STATS) {
+            float* o = p.stats_out + (size_t)gm * 8;
+            o[0] = M2;
+            o[1] = L;
+            o[2] = zyv;
+            o[3] = szv;
+            o[4] = __int_as_float(am);
+            return;
+        }
+    } else {
+        // every shard's statistics, merged in shard order (split softmax:
+        // lse = M + log2 sum_r l_r 2^(m_r - M); the target logit and the
+        // logit sums add over shards; ties go to the lowest shard)
+        int rbest = 0;
+        for (int r = 0; r < p.n_shards; ++r) {
+            const float v = p.all_stats[((size_t)r * p.stats_N + gm) * 8];
+            if (v > M2) { M2 = v; rbest = r; }
+        }
+        for (int r = 0; r < p.n_shards; ++r) {
+            const float* st = p.all_stats + ((size_t)r * p.stats_N + gm) * 8;
+            L += st[1] * exp2f(st[0] - M2);
+            zyv += st[2];
+            szv += st[3];
+        }
+        am = __float_as_int(p.all_stats[((size_t)rbest * p.stats_N + gm) * 8 + 4]);
     }
     const float lse2 = M2 + log2f(L);
     const float lse = lse2 * 0.69314718055994530942f;
-    const int64_t y = p.target[m];
-    const bool valid = (y != p.ignore_index) && y >= 0 && y < p.V;
     float loss = 0.f, gcoef = 0.f;
     if (valid) {
         const float T = p.total > 0.f ? p.total
                         : (float)(p.count_dev != nullptr ? *p.count_dev : p.cnt->n_valid);
         const float pm = p.p_mask != nullptr ? p.p_mask[m] : 1.f;
         const float coef = 1.f / (pm * T);
-        float ce = lse - p.zy[m];
-        if (p.eps > 0.f) {
-            float sz = 0.f;
-            for (int k = 0; k < p.n_vt; ++k) sz += p.part_sz[(size_t)k * p.ld_part + m];
-            const float meanz = p.s * sz / (float)p.V;
-            ce = (1.f - p.eps) * ce + p.eps * (lse - meanz);
-        }
+        float ce = lse - zyv;
+        if (p.eps > 0.f) ce = (1.f - p.eps) * ce + p.eps * (lse - szv / (float)p.Vtot);
         loss = ce * coef;
         gcoef = p.grad_out * p.s * coef;
     }
     p.loss_tok[m] = loss;
     if (p.lse_out != nullptr) p.lse_out[m] = lse;
-    if (p.am_out != nullptr) p.am_out[m] = p.part_am[(size_t)kbest * p.ld_part + m];
+    if (p.am_out != nullptr) p.am_out[m] = am;
     if (p.row_lse2 != nullptr) {
         p.row_lse2[m] = lse2;
         p.row_gcoef[m] = gcoef;
-        p.row_y[m] = valid ? (int32_t)y : -1;
+        p.row_y[m] = local_y ? (int32_t)(y - p.v0) : -1;
     }
 }
 
@@ -719,7 +761,7 @@ struct SimtLse {
         p.part_ml[o] = make_float2(mx, l);
         if (p.part_sz != nullptr) p.part_sz[o] = sz;
         if (p.part_am != nullptr) p.part_am[o] = (int32_t)(n0 + am);
-        const int64_t y = p.target[m];
+        const int64_t y = p.target[m] - p.v0;
         if (y >= n0 && y < n0 + ncols) p.zy[m] = C[r][y - n0] * p.s;
     }
 };

@@ -80,3 +80,64 @@ def fwd_bwd_data_parallel(kernels, H, W, target, p_mask, *, total: float = 0.0,
     kernels.reduce_weight_grads(grads, group)
     dist.all_reduce(out["loss"], op=dist.ReduceOp.SUM, group=group)
     return out
+
+
+# ---------------------------------------------------------------- vocabulary parallel
+
+class LibraryShardKernels:
+    """The per-rank steps of the vocabulary-parallel loss, through the C ABI.
+
+    ``plan`` must cover this rank's vocabulary shard (made with vocab_start /
+    vocab_total) and all tokens of the batch."""
+
+    def __init__(self, plan: B.Plan):
+        self.plan = plan
+
+    def vp_stats(self, H, W, target, p_mask, bias):
+        stats = torch.empty(H.shape[0], 8, dtype=torch.float32, device=self.plan.device)
+        call = B.make_call(H=H, W=W, bias=bias, target=target, p_mask=p_mask, N=H.shape[0],
+                           workspace=self.plan.workspace,
+                           workspace_bytes=self.plan.workspace_bytes)
+        B.fldce_vp_stats(self.plan.handle, call, stats)
+        return stats
+
+    def vp_fwd_bwd(self, H, W, target, p_mask, total, grad_out, bias, all_stats, out):
+        N = H.shape[0]
+        if out is None:
+            out = self.plan.outputs(N)
+            if bias is not None:
+                out["db"] = torch.empty_like(bias)
+        call = B.make_call(H=H, W=W, bias=bias, target=target, p_mask=p_mask, N=N,
+                           total=float(total), grad_out=float(grad_out), loss=out["loss"],
+                           loss_per_token=out.get("loss_per_token"), lse=out.get("lse"),
+                           argmax=out.get("argmax"), dH=out["dH"], dW=out["dW"],
+                           db=out.get("db"), workspace=self.plan.workspace,
+                           workspace_bytes=self.plan.workspace_bytes, err_count=out["err"])
+        B.fldce_vp_fwd_bwd(self.plan.handle, call, all_stats, all_stats.shape[0])
+        return out
+
+
+def fwd_bwd_vocab_parallel(kernels, H, W_shard, target, p_mask, *, total: float = 0.0,
+                           grad_out: float = 1.0, bias_shard=None, out: Optional[dict] = None,
+                           group=None) -> dict:
+    """One vocabulary-parallel step (the tensor-parallel tutorial page, section 4).
+
+    Every rank holds all tokens (H, target, p_mask) and the rows of W (and
+    bias) of its vocabulary shard; ranks are ordered by vocabulary offset.
+    1. each rank's sweep 1 writes per-token shard statistics (max, sum-exp,
+       target logit, logit sum, argmax): 32 bytes per token;
+    2. the statistics are all-gathered; every rank merges them in rank order
+       into the same lse and loss, and forms G for its own columns, giving
+       its dW and db shard and its partial dH;
+    3. the partial dH are summed across ranks.
+    Returns this rank's outputs: loss (the job's), dH (summed), dW / db (the
+    shard's).  Every rank holds all tokens, so the count normaliser is local.
+    """
+    stats = kernels.vp_stats(H, W_shard, target, p_mask, bias_shard)
+    P = dist.get_world_size(group)
+    all_stats = torch.empty((P,) + tuple(stats.shape), dtype=stats.dtype, device=stats.device)
+    dist.all_gather([all_stats[r] for r in range(P)], stats.contiguous(), group=group)
+    out = kernels.vp_fwd_bwd(H, W_shard, target, p_mask, total, grad_out, bias_shard,
+                             all_stats, out)
+    dist.all_reduce(out["dH"], op=dist.ReduceOp.SUM, group=group)
+    return out
