@@ -47,6 +47,8 @@ SMALL = [
     (77, 64, 40, {"grad_out": 2.5}),
     (5, 8, 300, {"total": 1.0}),
     (513, 520, 2049, {"label_smoothing": 0.3, "logit_scale": 1.7, "grad_out": -0.75}),
+    (1, 64, 1000, {}),
+    (200, 64, 1000, {"logit_scale": -0.7, "label_smoothing": 0.1}),
 ]
 
 
@@ -171,3 +173,16 @@ def test_error_codes_leave_outputs_untouched():
                         None, None, out["dH"].data_ptr() + 2, out["dW"], plan.workspace,
                         plan.workspace_bytes, None)
     assert e.value.status == B.FLDCE_ERR_ALIGN
+
+
+def test_ignore_index_inside_vocabulary():
+    """ignore_index may be a real vocabulary id (here 0): those targets carry
+    no loss, and nothing else changes."""
+    wl = _small(300, 64, 500, seed=12)
+    t = wl.target.clone()
+    t[t == -100] = 0
+    t[3::7] = 0
+    wl.target = t
+    wl.ignore_index = 0
+    g = run_gpu(wl)
+    _full_compare(wl, g, "bf16")
