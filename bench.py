@@ -211,6 +211,8 @@ def main():
                     help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--compare-cublas", action="store_true",
+                    help="also time torch.matmul (cuBLAS) on the step's three GEMM shapes")
     ap.add_argument("--no-skip", action="store_true",
                     help="do not time the FLDCE_FLAG_SKIP_IGNORED variant")
     args = ap.parse_args()
@@ -349,6 +351,10 @@ def main():
         splan.close()
         del sout
 
+    cublas = None
+    if args.compare_cublas and world == 1 and wl.H.dtype == torch.bfloat16:
+        cublas = time_cublas_same_shapes(H, W, args.steps, dev, stream)
+
     e2e = None
     if not args.no_e2e:
         if dist is None:
@@ -380,12 +386,40 @@ def main():
             "kernel_share": {k: v[0] / total_kernel_ms for k, v in kinds.items()},
             "gpu_launches": launches,
             "skip_ignored": skip,
+            "cublas_same_shapes": cublas,
             "e2e": e2e, "cpu_baseline": cb, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def time_cublas_same_shapes(H, W, steps, dev, stream):
+    """torch.matmul (cuBLAS) on the three GEMM shapes of one step, as a
+    reference point for the fused kernels: logits H W^T [N,V] (written out,
+    unlike sweep 1), dH = G W and dW = G^T H with a random bf16 G [N,V]."""
+    N, D = H.shape
+    V = W.shape[0]
+    G = (torch.randn(N, V, device=dev) * 1e-4).bfloat16()
+    res = {}
+    for name, fn in (("logits", lambda: H @ W.t()), ("dH", lambda: G @ W),
+                     ("dW", lambda: G.t() @ H)):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        k = max(3, min(steps, 10))
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / k
+        res[name] = {"ms": ms, "tflops": 2.0 * N * D * V / (ms / 1e3) / 1e12}
+    del G
+    return res
 
 
 def traffic_for(kernel: str, workload: str):

@@ -256,7 +256,7 @@ int fldce_forward_ex(fldce_handle h, const fldce_call* call);
  *
  * fldce_vp_stats -- sweep 1 over this shard: for each token n, 8 fp32 at
  *   stats[8 n .. 8 n + 7]: m2 (max of z log2 e over the shard), l (sum of
- *   2^(z log2 e - m2)), z[n, y_n] if y_n is in the shard else 0, s * sum of
+ *   2^(z log2 e - m2)), z[n, y_n] log2 e if y_n is in the shard else 0, s * sum of
  *   (H W^T + b) over the shard, the shard argmax as int32 bits (global id),
  *   3 unused.  Uses call->H, W, bias, target, N, workspace, stream.
  *   stats [device, out] [N][8] fp32.

@@ -87,7 +87,7 @@ struct LseEpi {
         float2* part_ml;         // [n_vt][ld_part] (m2, l)
         float* part_sz;          // [n_vt][ld_part] sum of acc, or null
         int32_t* part_am;        // [n_vt][ld_part] argmax column, or null
-        float* zy;               // [ld_part] target logit z[n, y_n]
+        float* zy;               // [ld_part] target logit z[n, y_n] log2(e)
         const __nv_bfloat16* bias;   // [V] or null
         int64_t v0;              // first vocabulary id of this shard (0 unsharded)
     };
@@ -169,7 +169,7 @@ struct LseEpi {
             p.part_ml[o] = make_float2(mx, l);
             if (want_sz) p.part_sz[o] = sz;
             if (want_am) p.part_am[o] = (int32_t)(n0 + am);
-            if (yrel >= 0) p.zy[m] = zyv * p.s;
+            if (yrel >= 0) p.zy[m] = zyv * p.c;    // base 2, rounded like the maxima
         }
     }
 };
@@ -579,7 +579,9 @@ __global__ void k_merge_rows(MergeParams p) {
                         : (float)(p.count_dev != nullptr ? *p.count_dev : p.cnt->n_valid);
         const float pm = p.p_mask != nullptr ? p.p_mask[m] : 1.f;
         const float coef = 1.f / (pm * T);
-        float ce = lse - zyv;
+        // lse - z_y taken in base 2, where both carry the same rounding of
+        // acc * s * log2(e) (exactly 0 when the target is the only column)
+        float ce = (lse2 - zyv) * 0.69314718055994530942f;
         if (p.eps > 0.f) ce = (1.f - p.eps) * ce + p.eps * (lse - szv / (float)p.Vtot);
         loss = ce * coef;
         gcoef = p.grad_out * p.s * coef;
@@ -762,7 +764,7 @@ struct SimtLse {
         if (p.part_sz != nullptr) p.part_sz[o] = sz;
         if (p.part_am != nullptr) p.part_am[o] = (int32_t)(n0 + am);
         const int64_t y = p.target[m] - p.v0;
-        if (y >= n0 && y < n0 + ncols) p.zy[m] = C[r][y - n0] * p.s;
+        if (y >= n0 && y < n0 + ncols) p.zy[m] = C[r][y - n0] * p.c;
     }
 };
 

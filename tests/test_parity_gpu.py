@@ -49,7 +49,18 @@ SMALL = [
     (513, 520, 2049, {"label_smoothing": 0.3, "logit_scale": 1.7, "grad_out": -0.75}),
     (1, 64, 1000, {}),
     (200, 64, 1000, {"logit_scale": -0.7, "label_smoothing": 0.1}),
+    (50, 64, 1, {}),
+    (96, 64, 500, {"label_smoothing": 1.0}),
 ]
+
+
+def test_large_logits():
+    """Logits in the hundreds (unit-scale W, logit_scale 30): the running
+    maxima keep every exponential finite."""
+    wl = _small(128, 64, 700, seed=13, sigma=1.0, logit_scale=30.0)
+    g = run_gpu(wl)
+    assert torch.isfinite(g["dH"].float()).all() and torch.isfinite(g["lse"]).all()
+    _full_compare(wl, g, "bf16")
 
 
 @pytest.mark.parametrize("N,D,V,kw", SMALL, ids=[f"N{a}_D{b}_V{c}" for a, b, c, _ in SMALL])
