@@ -396,28 +396,37 @@ def main():
 
 
 def time_cublas_same_shapes(H, W, steps, dev, stream):
-    """torch.matmul (cuBLAS) on the three GEMM shapes of one step, as a
-    reference point for the fused kernels: logits H W^T [N,V] (written out,
-    unlike sweep 1), dH = G W and dW = G^T H with a random bf16 G [N,V]."""
+    """torch.matmul (cuBLAS) on the GEMM shapes of one step, as a reference
+    point for the fused kernels: a "cuBLAS step" of logits H W^T [N,V] twice
+    (written out, unlike the sweeps), dH = G W and dW = G^T H with a random
+    bf16 G [N,V], run back to back for as many steps as the timed loop so
+    both see the same power-capped clock."""
     N, D = H.shape
     V = W.shape[0]
     G = (torch.randn(N, V, device=dev) * 1e-4).bfloat16()
+    gemms = (("logits", lambda: H @ W.t()), ("logits", lambda: H @ W.t()),
+             ("dH", lambda: G @ W), ("dW", lambda: G.t() @ H))
+    for _, fn in gemms:
+        fn()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(gemms) + 1)]
+          for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record(stream)
+        for i, (_, fn) in enumerate(gemms):
+            fn()
+            ev[k][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
     res = {}
-    for name, fn in (("logits", lambda: H @ W.t()), ("dH", lambda: G @ W),
-                     ("dW", lambda: G.t() @ H)):
-        for _ in range(2):
-            fn()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        k = max(3, min(steps, 10))
-        e0.record(stream)
-        for _ in range(k):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / k
-        res[name] = {"ms": ms, "tflops": 2.0 * N * D * V / (ms / 1e3) / 1e12}
+    for i, (name, _) in enumerate(gemms):
+        ms = sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
+        r = res.setdefault(name, {"ms": 0.0, "n": 0})
+        r["ms"] += ms
+        r["n"] += 1
+    for r in res.values():
+        r["ms"] /= r.pop("n")
+        r["tflops"] = 2.0 * N * D * V / (r["ms"] / 1e3) / 1e12
+    res["step_ms"] = sum(ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps)) / steps
     del G
     return res
 
