@@ -492,7 +492,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
         mp.row_lse2 = backward && mode != MERGE_EMIT_STATS ? row_lse2 : nullptr;
         mp.row_gcoef = row_gcoef;
         mp.row_y = row_y;
-        k_merge_rows<<<(unsigned)cdiv(rows, 128), 128, 0, st>>>(mp);
+        k_merge_rows<<<(unsigned)cdiv((int64_t)rows * kMergeSub, 256), 256, 0, st>>>(mp);
         FLDCE_CUDA(cudaGetLastError());
         prof_mark(h, PK_MERGE, st);
         if (!backward || mode == MERGE_EMIT_STATS) continue;

@@ -508,10 +508,54 @@ struct MergeParams {
 // logsumexp; the tensor-parallel tutorial's sum of per-shard denominators),
 // then the per-token loss (cross_entropy_kernel step 4 and the
 // label-smoothing block) and the per-token gradient coefficient.
-__global__ void k_merge_rows(MergeParams p) {
-    const int m = blockIdx.x * blockDim.x + threadIdx.x;
-    if (m >= p.rows) return;
-    if (p.dyn_count != nullptr && m >= *p.dyn_count - p.dyn_base) {
+// Threads per row of the split-V merge: each takes every kMergeSub-th vocab
+// tile in one online pass; the kMergeSub partial (max, sum) pairs of a row are
+// then combined with shuffles in a fixed order (deterministic).
+constexpr int kMergeSub = 8;
+
+__global__ void __launch_bounds__(256) k_merge_rows(MergeParams p) {
+    const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+    const int m = tid / kMergeSub;
+    const int g = tid % kMergeSub;
+    bool live = m < p.rows;
+    bool dead_dyn = false;
+    if (live && p.dyn_count != nullptr && m >= *p.dyn_count - p.dyn_base) {
+        live = false;
+        dead_dyn = true;
+    }
+    const int64_t gm = p.stats_row0 + m;          // token index within the call
+    float M2 = -CUDART_INF_F, L = 0.f, szs = 0.f;
+    int kbest = 0x7fffffff;
+    if (live && p.mode != MERGE_GATHERED) {
+        for (int k = g; k < p.n_vt; k += kMergeSub) {
+            const float2 ml = p.part_ml[(size_t)k * p.ld_part + m];
+            if (ml.x > M2) {
+                L = L * exp2f(M2 - ml.x) + ml.y;
+                M2 = ml.x;
+                kbest = k;
+            } else {
+                L += ml.y * exp2f(ml.x - M2);
+            }
+            if (p.part_sz != nullptr) szs += p.part_sz[(size_t)k * p.ld_part + m];
+        }
+    }
+    // combine the kMergeSub lanes of the row (all lanes take part)
+#pragma unroll
+    for (int o = 1; o < kMergeSub; o <<= 1) {
+        const float Mo = __shfl_xor_sync(0xffffffffu, M2, o);
+        const float Lo = __shfl_xor_sync(0xffffffffu, L, o);
+        const int ko = __shfl_xor_sync(0xffffffffu, kbest, o);
+        const float so = __shfl_xor_sync(0xffffffffu, szs, o);
+        const float Mn = fmaxf(M2, Mo);
+        const float a = (M2 == -CUDART_INF_F) ? 0.f : L * exp2f(M2 - Mn);
+        const float b = (Mo == -CUDART_INF_F) ? 0.f : Lo * exp2f(Mo - Mn);
+        kbest = (Mo > M2 || (Mo == M2 && ko < kbest)) ? ko : kbest;
+        L = a + b;
+        M2 = Mn;
+        szs += so;
+    }
+    if (g != 0 || m >= p.rows) return;
+    if (dead_dyn) {
         // past the compacted tokens: no loss, zero gradient row
         p.loss_tok[m] = 0.f;
         if (p.row_lse2 != nullptr) {
@@ -521,29 +565,14 @@ __global__ void k_merge_rows(MergeParams p) {
         }
         return;
     }
-    const int64_t gm = p.stats_row0 + m;          // token index within the call
     const int64_t y = p.target[m];
     const bool valid = (y != p.ignore_index) && y >= 0 && y < p.Vtot;
     const bool local_y = valid && y - p.v0 >= 0 && y - p.v0 < p.V;
-    float M2 = -CUDART_INF_F, L = 0.f, zyv = 0.f, szv = 0.f;
+    float zyv = 0.f, szv = 0.f;
     int32_t am = -1;
     if (p.mode != MERGE_GATHERED) {
-        // this shard's vocab tiles
-        int kbest = 0;
-        for (int k = 0; k < p.n_vt; ++k) {
-            const float v = p.part_ml[(size_t)k * p.ld_part + m].x;
-            if (v > M2) { M2 = v; kbest = k; }
-        }
-        for (int k = 0; k < p.n_vt; ++k) {
-            const float2 ml = p.part_ml[(size_t)k * p.ld_part + m];
-            L += ml.y * exp2f(ml.x - M2);
-        }
         if (local_y) zyv = p.zy[m];
-        if (p.part_sz != nullptr) {
-            float sz = 0.f;
-            for (int k = 0; k < p.n_vt; ++k) sz += p.part_sz[(size_t)k * p.ld_part + m];
-            szv = p.s * sz;
-        }
+        szv = p.s * szs;
         if (p.part_am != nullptr) am = p.part_am[(size_t)kbest * p.ld_part + m] + (int32_t)p.v0;
         if (p.mode == MERGE_EMIT_STATS) {
             float* o = p.stats_out + (size_t)gm * 8;
