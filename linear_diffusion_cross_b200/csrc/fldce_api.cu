@@ -1,14 +1,21 @@
 // fldce_api.cu -- host side of the C ABI declared in include/fldce.h.
 //
-// One call runs, on the caller's stream and without any host synchronisation:
-//   k_count_targets                      all N tokens (the normaliser T)
+// One fwd+bwd call enqueues, on the caller's stream and without any host
+// synchronisation:
+//   k_count_targets                  all N tokens (the normaliser T, bad targets)
+//   [SKIP_IGNORED] k_compact_valid, k_gather_rows   compact the valid tokens
 //   per token chunk [r0, r0 + rows):
-//     sweep 1  GEMM H W^T + LseEpi       per (row, vocab tile) partial lse
-//     k_merge_rows                       lse, loss[n], gradient coefficient
-//     sweep 2  GEMM H W^T + GEpi         G (bf16) for the chunk
-//     dH GEMM  G W                       dH rows of the chunk
-//     dW GEMM  G^T H                     dW (accumulated over chunks)
-//   k_finish                             fixed-order loss sum, error count
+//     sweep 1  GEMM H W^T (+b), LseEpi      per (row, vocab tile) partial lse
+//     k_merge_rows                          lse, loss[n], gradient coefficient
+//     sweep 2  GEMM H W^T (+b), GEpi        G (bf16) for the chunk
+//     [bias] k_colsum_*                     db (+)= column sums of G
+//     dH GEMM  G W       (+ k_f32_to_bf16 when the vocabulary is split in two)
+//     dW GEMM  G^T H     (fp32 across chunks, converted after the last)
+//   [SKIP_IGNORED] k_scatter_rows       dH and per-token outputs back in place
+//   k_finish                             fixed-order loss sum, error counts
+// The vocabulary-parallel entry points run the same pipeline on one shard of
+// W: fldce_vp_stats stops after sweep 1 and writes the shard's per-token
+// statistics; fldce_vp_fwd_bwd skips sweep 1 and merges every shard's.
 // The chunk loop is the page's fused_linear_cross_entropy_forward loop over
 // token chunks; it bounds the workspace.  bf16 runs on tcgen05 tensor cores;
 // fp32 runs the CUDA-core GEMM of kernels.cuh.
@@ -49,16 +56,26 @@ struct DeviceInfo {
     int sms = 0;
 };
 
+// Compute capability and SM count of the current device (cached per device;
+// calls may come from several host threads).
 bool device_info(DeviceInfo* out) {
+    static std::mutex mu;
     static DeviceInfo cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
-    if (dev < 64 && cache[dev].major >= 0) { *out = cache[dev]; return true; }
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 64 && cache[dev].major >= 0) {
+            *out = cache[dev];
+            return true;
+        }
+    }
     DeviceInfo d;
     if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
         return false;
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return false;
+    std::lock_guard<std::mutex> lock(mu);
     if (dev < 64) cache[dev] = d;
     *out = d;
     return true;
@@ -69,16 +86,18 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's cuTensorMapEncodeTiled, looked up once (no link-time libcuda).
 EncodeTiledFn encode_fn() {
+    static std::once_flag once;
     static EncodeTiledFn fn = nullptr;
-    if (fn == nullptr) {
+    std::call_once(once, [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
+    });
     return fn;
 }
 
