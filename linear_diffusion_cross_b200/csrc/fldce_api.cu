@@ -9,7 +9,7 @@
 //     k_merge_rows                          lse, loss[n], gradient coefficient
 //     sweep 2  GEMM H W^T (+b), GEpi        G (bf16) for the chunk
 //     [bias] k_colsum_*                     db (+)= column sums of G
-//     dH GEMM  G W       (+ k_f32_to_bf16 when the vocabulary is split in two)
+//     dH GEMM  G W       (+ k_sum_splits when the vocabulary is split in k ranges)
 //     dW GEMM  G^T H     (fp32 across chunks, converted after the last)
 //   [SKIP_IGNORED] k_scatter_rows       dH and per-token outputs back in place
 //   k_finish                             fixed-order loss sum, error counts
@@ -42,6 +42,7 @@ constexpr int kBN = 256;               // vocab tile of the tensor-core sweeps
 constexpr int kStages = 6;
 constexpr size_t kAlign = 256;
 constexpr size_t kGBudget = size_t(1) << 32;   // G buffer per chunk: at most 4 GiB
+constexpr int kMaxKSplits = 4;                  // K splits of the dH GEMM
 constexpr int kColsumSegs = 8;                  // row segments of the db column sums
 
 using CfgKK = GemmCfg<kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
@@ -126,10 +127,17 @@ bool make_store_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
     return make_map(m, base, cols, rows, ld, elt == 4 ? 32 : 64, 32, elt);
 }
 
-// Units (tiles x K splits) per pair round; the fraction of pair slots busy.
-double wave_efficiency(int64_t units, int pairs) {
-    const int64_t rounds = (units + pairs - 1) / pairs;
-    return rounds == 0 ? 1.0 : (double)units / (double)(rounds * pairs);
+// K splits of a GEMM with `tiles` output tiles and `k_iters` K steps on
+// `pairs` CTA pairs.  The persistent schedule runs ceil(k tiles / pairs)
+// rounds of ceil(k_iters / k) steps; a split is taken only when it shortens
+// that by more than 2% (each split costs an fp32 partial buffer and its
+// share of the fixed-order sum) and keeps >= 16 K steps per split.
+int choose_k_splits(int64_t tiles, int64_t k_iters, int pairs) {
+    auto cost = [&](int64_t k) { return cdiv(k * tiles, pairs) * cdiv(k_iters, k); };
+    int best = 1;
+    for (int k = 2; k <= kMaxKSplits; ++k)
+        if (k_iters >= 16 * k && (double)cost(k) < 0.98 * (double)cost(best)) best = k;
+    return best;
 }
 
 struct DynRows {
@@ -178,6 +186,20 @@ cudaError_t launch_colsum(const void* G, bool g_bf16, int64_t ldg, int rows, int
         k_colsum_partial<float><<<grid, 128, 0, st>>>(static_cast<const float*>(G), ldg, rows, V,
                                                       seg_rows, part, dyn_count, dyn_base);
     k_colsum_final<<<(unsigned)cdiv(V, 256), 256, 0, st>>>(part, nseg, V, acc, add ? 1 : 0);
+    return cudaGetLastError();
+}
+
+// dst = sum of k fp32 partials `stride` floats apart (bf16 or fp32 out).
+cudaError_t launch_sum_splits(const float* part, int64_t stride, int k, void* dst, bool to_bf16,
+                              int64_t n, int sms, cudaStream_t st) {
+    const int64_t n8 = n / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(cdiv(n8, 256), 8 * (int64_t)sms);
+    if (to_bf16)
+        k_sum_splits<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+            part, stride, k, static_cast<__nv_bfloat16*>(dst), n8);
+    else
+        k_sum_splits<float><<<blocks, 256, 0, st>>>(part, stride, k, static_cast<float*>(dst), n8);
     return cudaGetLastError();
 }
 
@@ -269,7 +291,10 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
     L.row_y = take(C * 4);
     L.loss_tok = take(std::max<int64_t>(N, 1) * 4);
     L.G = take((size_t)C * p->Vpad * p->elt);
-    L.dh_acc = take(p->cfg.dtype == FLDCE_BF16 ? (size_t)C * p->cfg.D * 4 : 0);
+    // one fp32 partial per K split of dH, each padded to whole pair tiles
+    L.dh_acc = take(p->cfg.dtype == FLDCE_BF16
+                        ? (size_t)kMaxKSplits * round_up((size_t)C, 256) * p->cfg.D * 4
+                        : 0);
     const bool acc = L.nchunks > 1 && !dw_out_fp32(p);
     L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
     L.db_part = take((size_t)kColsumSegs * p->cfg.V * 4);
@@ -557,37 +582,37 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             if (!make_map(&mH_mn, Hc, D, rows, D, 64, 64)) return FLDCE_ERR_CUDA;
 
             // dH = G W (K = V).  When one pass over the tiles leaves many SMs
-            // idle in its last round, the vocabulary is split in two halves
-            // whose fp32 partials are reduce-added into a zeroed buffer (two
-            // addends: the sum does not depend on their order).
+            // idle in its last round, the vocabulary is split into k ranges;
+            // split j stores its fp32 partial in its own buffer and one pass
+            // sums them in split order (deterministic) into dH.
             auto do_dh = [&]() -> int {
-                const int pairs = std::max(1, dev.sms / 2);
                 const int64_t dh_tiles = cdiv(rows, CfgKM::PAIR_M) * cdiv(D, CfgKM::BN);
-                const bool dh_split = cdiv(V, CfgKM::BK) >= 8 &&
-                                      wave_efficiency(2 * dh_tiles, pairs) >
-                                          wave_efficiency(dh_tiles, pairs) + 0.03;
+                const int ks = choose_k_splits(dh_tiles, cdiv(V, CfgKM::BK),
+                                               std::max(1, dev.sms / 2));
                 StoreEpi::Params hp;
                 const bool dh_fp32 = (cfg.flags & FLDCE_FLAG_DH_FP32) != 0;
-                float* dh_acc = dh_fp32 ? static_cast<float*>(dH) + r0 * D
-                                        : reinterpret_cast<float*>(ws + L.dh_acc);
-                void* dHc = static_cast<__nv_bfloat16*>(dH) + r0 * D;
-                if (dh_split) {
-                    FLDCE_CUDA(cudaMemsetAsync(dh_acc, 0, (size_t)rows * D * 4, st));
-                    if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
-                    hp.mode = WS_ADD;
+                float* part = reinterpret_cast<float*>(ws + L.dh_acc);
+                const int split_rows = (int)round_up((size_t)rows, 256);
+                void* dHc = static_cast<uint8_t*>(dH) + (size_t)r0 * D * (dh_fp32 ? 4 : 2);
+                if (ks > 1) {
+                    if (!make_store_map(&hp.omap, part, D, (uint64_t)ks * split_rows, D, 4))
+                        return FLDCE_ERR_CUDA;
+                    hp.mode = WS_STORE;
+                    hp.split_rows = split_rows;
                 } else if (dh_fp32) {
-                    if (!make_store_map(&hp.omap, dh_acc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
+                    if (!make_store_map(&hp.omap, dHc, D, rows, D, 4)) return FLDCE_ERR_CUDA;
                     hp.mode = WS_STORE;
                 } else {
                     if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
                     hp.mode = OUT_BF16;
                 }
-                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1,
-                                                         dh_split ? 2 : 1, hp, &cnt->dev_err,
-                                                         dev.sms, st, DynRows{dynp, (int)r0, 1})));
+                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1, ks, hp,
+                                                         &cnt->dev_err, dev.sms, st,
+                                                         DynRows{dynp, (int)r0, 1})));
                 prof_mark(h, PK_DH, st);
-                if (dh_split && !dh_fp32) {
-                    FLDCE_CUDA(launch_to_bf16(dh_acc, dHc, (int64_t)rows * D, dev.sms, st));
+                if (ks > 1) {
+                    FLDCE_CUDA(launch_sum_splits(part, (int64_t)split_rows * D, ks, dHc,
+                                                 !dh_fp32, (int64_t)rows * D, dev.sms, st));
                     prof_mark(h, PK_CONVERT, st);
                 }
                 return FLDCE_OK;
@@ -712,8 +737,10 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
     p->n_vt = cdiv(cfg->V, p->tile_v);
     int64_t chunk = cfg->chunk_N;
     if (chunk == 0) {
-        chunk = (int64_t)(kGBudget / ((size_t)p->Vpad * p->elt)) / 128 * 128;
-        chunk = std::max<int64_t>(chunk, 128);
+        // whole 256-row pair tiles, so no chunk but the last ends in a
+        // partly empty M tile
+        chunk = (int64_t)(kGBudget / ((size_t)p->Vpad * p->elt)) / 256 * 256;
+        chunk = std::max<int64_t>(chunk, 256);
     }
     p->chunk = std::min<int64_t>(chunk, cfg->max_N);
     if (workspace_bytes != nullptr) *workspace_bytes = make_layout(p, cfg->max_N).total;

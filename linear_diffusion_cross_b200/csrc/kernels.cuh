@@ -280,7 +280,10 @@ struct GEpi {
 // Epilogue 3: dH / dW tiles.
 //   OUT_BF16: bf16 output, 64-column boxes, TMA store;
 //   WS_STORE / WS_ADD: fp32 32-column boxes, TMA store or TMA reduce-add
-//   (dW accumulated over token chunks; dH split over two vocab halves).
+//   (dW accumulated over token chunks).
+// A GEMM split over K (dH over vocabulary ranges) stores split j's tile
+// split_rows * j rows further down, so every split owns a partial buffer
+// that a later pass sums in a fixed order.
 // ======================================================================
 enum StoreMode { OUT_BF16 = 0, WS_STORE = 1, WS_ADD = 2 };
 
@@ -288,13 +291,14 @@ struct StoreEpi {
     struct Params {
         CUtensorMap omap;        // bf16 [rows, cols] box 64 x 32, or fp32 box 32 x 32
         int mode;
+        int split_rows = 0;      // row offset between K splits' partial buffers
     };
 
     template <class Cfg>
     static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
                                                const AccRow& acc, Stager& st) {
         const int64_t n0 = t.col0;
-        const int y = t.row0 + 32 * t.q;
+        const int y = t.row0 + t.split * p.split_rows + 32 * t.q;
         const int mode = p.mode;
         for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
             if (mode == OUT_BF16) {
@@ -661,6 +665,36 @@ __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __re
         w.z = pack_bf16x2(b.x, b.y);
         w.w = pack_bf16x2(b.z, b.w);
         reinterpret_cast<uint4*>(dst)[i] = w;
+    }
+}
+
+// out[i] = sum_j part[j * stride + i], j = 0 .. k-1 in that order (the K
+// splits of one GEMM), so the result does not depend on which split
+// finished first.  n8 = elements / 8.
+template <class OutT>
+__global__ void k_sum_splits(const float* __restrict__ part, int64_t stride, int k,
+                             OutT* __restrict__ out, int64_t n8) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = reinterpret_cast<const float4*>(part)[2 * i];
+        float4 b = reinterpret_cast<const float4*>(part)[2 * i + 1];
+        for (int j = 1; j < k; ++j) {
+            const float4* q = reinterpret_cast<const float4*>(part + j * stride);
+            const float4 c = q[2 * i], d = q[2 * i + 1];
+            a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+            b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+        }
+        if constexpr (sizeof(OutT) == 2) {
+            uint4 w;
+            w.x = pack_bf16x2(a.x, a.y);
+            w.y = pack_bf16x2(a.z, a.w);
+            w.z = pack_bf16x2(b.x, b.y);
+            w.w = pack_bf16x2(b.z, b.w);
+            reinterpret_cast<uint4*>(out)[i] = w;
+        } else {
+            reinterpret_cast<float4*>(out)[2 * i] = a;
+            reinterpret_cast<float4*>(out)[2 * i + 1] = b;
+        }
     }
 }
 

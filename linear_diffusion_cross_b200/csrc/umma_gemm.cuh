@@ -70,7 +70,7 @@ struct GemmGeom {
     int tiles_m;          // ceil(M / 256)
     int tiles_n;          // ceil(N / 256)
     int k_iters;          // ceil(K / 64)
-    int k_splits;         // K ranges per tile (1 or 2)
+    int k_splits;         // K ranges per tile (1 to 4)
     int num_tiles;        // tiles_m * tiles_n
     int n_fastest;        // 1: consecutive tiles walk n first (share the A panel)
     // Optional row count known only on the device (compacted tokens): the

@@ -34,13 +34,14 @@ def maxabs_err(got: np.ndarray, ref: np.ndarray) -> float:
 
 
 def run_gpu(wl: Workload, *, chunk_n=None, want_argmax=True, dw_fp32=False, p_mask_none=False,
-            plan=None, max_N=None):
+            plan=None, max_N=None, dh_fp32=False):
     dev = torch.device("cuda")
     if plan is None:
         plan = B.Plan(wl.D, wl.V, max_N or max(wl.N, 1), dtype=wl.H.dtype,
                       chunk_N=wl.chunk_n if chunk_n is None else chunk_n,
                       logit_scale=wl.logit_scale, label_smoothing=wl.label_smoothing,
-                      ignore_index=wl.ignore_index, dw_fp32=dw_fp32, device=dev)
+                      ignore_index=wl.ignore_index, dw_fp32=dw_fp32, dh_fp32=dh_fp32,
+                      device=dev)
     H = wl.H.to(dev)
     W = wl.W.to(dev)
     y = wl.target.to(dev)

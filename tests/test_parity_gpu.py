@@ -197,3 +197,18 @@ def test_ignore_index_inside_vocabulary():
     wl.ignore_index = 0
     g = run_gpu(wl)
     _full_compare(wl, g, "bf16")
+
+
+# dH's vocabulary reduction is split into k ranges when that fills the last
+# round of CTA pairs better: with 2 token tiles x 1 column tile, V = 3500 (55
+# K steps) takes 3 splits and V = 5003 (79 K steps) takes 4.  Each split's
+# fp32 partial is summed in split order, so dH is also bit-reproducible.
+@pytest.mark.parametrize("V", [3500, 5003])
+@pytest.mark.parametrize("dh_fp32", [False, True])
+def test_split_dh(V, dh_fp32):
+    wl = _small(300, 136, V, seed=14, label_smoothing=0.05)
+    g = run_gpu(wl, dh_fp32=dh_fp32)
+    assert g["dH"].dtype == (torch.float32 if dh_fp32 else torch.bfloat16)
+    _full_compare(wl, g, "bf16")
+    g2 = run_gpu(wl, plan=g["plan"])
+    assert torch.equal(g["dH"], g2["dH"])
