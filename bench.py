@@ -26,6 +26,7 @@ float64 oracle (the reference arm of this comparison) on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -68,11 +69,13 @@ def workload_desc(name: str, r: synth.Recipe) -> str:
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples every 200 ms while running."""
+    """nvidia-smi clock / throttle samples every 50 ms while running; the
+    summary keeps the samples stamped inside the timed window."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
@@ -84,7 +87,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -95,13 +98,22 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
+            if len(parts) >= 10:
                 self.rows.append(parts)
 
-    def stop(self):
+    @staticmethod
+    def _stamp(ts: str):
+        try:
+            return datetime.datetime.strptime(ts, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
+    def stop(self, t0: float, t1: float):
+        """Summary of the samples stamped in [t0, t1] (host epoch seconds);
+        all samples when none fall inside."""
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -111,14 +123,26 @@ class ClockSampler:
             self.thread.join(timeout=2)
         if not self.rows:
             return None
-        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4)
-                          if r[5 + i].lower().startswith("active")})
+        inside = [r for r in self.rows
+                  if (ts := self._stamp(r[0])) is not None and t0 <= ts <= t1]
+        rows = inside or self.rows
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [v for r in rows if (v := num(r[2])) is not None]
+        mx = [v for r in rows if (v := num(r[3])) is not None]
+        pw = [v for r in rows if (v := num(r[4])) is not None]
+        reasons = sorted({self.NAMES[i] for r in rows for i in range(4)
+                          if r[6 + i].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "power_w": statistics.median(pw) if pw else None,
+                "reasons": reasons, "samples": len(rows),
+                "window": "timed region" if inside else "whole sampler run"}
 
 
 _W64 = {}
@@ -157,7 +181,6 @@ def dist_setup(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and args.impl == "fldce":
-        import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
@@ -275,13 +298,15 @@ def main():
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
+    t_start = time.time()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    t_end = time.time()
     barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_start, t_end)
     prof = B.fldce_profile_end(plan.handle)
     ms_total = ev0.elapsed_time(ev1)
     if dist is not None:
@@ -368,15 +393,21 @@ def main():
         cb.pop("seconds", None)
 
     if rank == 0:
+        w_mb = V * D * wl.W.element_size() / 1e6
+        l2_note = (f"inputs larger than L2 (W is {w_mb:.0f} MB, L2 126 MB); no flush"
+                   if w_mb > 126 else
+                   f"inputs fit in L2 (W is {w_mb:.1f} MB); not flushed: a parity-size "
+                   "workload, not the headline line")
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.H.dtype == torch.bfloat16 else "f32",
             "data": "synthetic (seeded; shapes and masking of the workload)",
             "config": {"workload": workload_desc(args.workload, r), "N": N, "D": D, "V": V,
                        "chunk_N": B.fldce_chunk_size(plan.handle),
                        "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (W is 778 MB, L2 126 MB); no flush"},
+                       "l2": l2_note},
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "tflops_executed_8NDV": world * flops * 4 / 3 / (ms / 1e3) / 1e12,
             "pct_of_bf16_peak": 100.0 * flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],

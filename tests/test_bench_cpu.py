@@ -1,0 +1,65 @@
+"""Host logic of bench.py that needs no GPU: the clock-sample summary keeps
+only the samples stamped inside the timed window, and the roofline traffic
+lookup refuses counters taken on other sources."""
+import datetime
+
+import bench
+
+
+class _Proc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _row(t, mhz, power, cap):
+    ts = datetime.datetime.fromtimestamp(t).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    return [ts, "0", str(mhz), "1965", str(power), "0x4" if cap else "0x0",
+            "Not Active", "Not Active", "Not Active", "Active" if cap else "Not Active"]
+
+
+def _sampler(rows):
+    s = bench.ClockSampler(0)
+    s.proc = _Proc()
+    s.rows = rows
+    return s
+
+
+def test_clock_summary_keeps_the_timed_window():
+    t0 = 1_800_000_000.0
+    rows = [_row(t0 - 0.2, 1965, 120, False), _row(t0 - 0.1, 1965, 130, False),
+            _row(t0 + 0.05, 1500, 990, True), _row(t0 + 0.10, 1410, 1000, True),
+            _row(t0 + 0.15, 1455, 995, True), _row(t0 + 0.5, 1965, 140, False)]
+    c = _sampler(rows).stop(t0, t0 + 0.2)
+    assert c["window"] == "timed region" and c["samples"] == 3
+    assert c["sm_mhz"] == 1455 and c["power_w"] == 995
+    assert c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_falls_back_to_all_samples():
+    t0 = 1_800_000_000.0
+    rows = [_row(t0 - 1.0, 1965, 120, False), _row(t0 + 1.0, 1900, 300, False)]
+    c = _sampler(rows).stop(t0, t0 + 0.01)
+    assert c["window"] == "whole sampler run" and c["samples"] == 2
+    assert c["reasons"] == []
+
+
+def test_traffic_needs_counters_of_the_current_sources():
+    # a kernel with no committed summary has no traffic figure
+    assert bench.traffic_for("no_such_kernel", "headline") is None
+
+
+def test_traffic_follows_the_source_hash(tmp_path, monkeypatch):
+    csrc = tmp_path / "linear_diffusion_cross_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("// v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_hash()
+    (tmp_path / "profiles" / "ncu_k_w.txt").write_text(
+        f"source_sha256: {h}\ndram_bytes_per_launch: 1.5e9\n")
+    assert bench.traffic_for("k", "w") == 1.5e9
+    (csrc / "k.cu").write_text("// v2\n")          # the kernel changed since the capture
+    assert bench.traffic_for("k", "w") is None
