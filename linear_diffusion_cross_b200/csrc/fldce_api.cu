@@ -26,6 +26,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <limits>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -43,6 +44,11 @@ constexpr int kStages = 6;
 constexpr size_t kAlign = 256;
 constexpr size_t kGBudget = size_t(1) << 32;   // G buffer per chunk: at most 4 GiB
 constexpr int kMaxKSplits = 4;                  // K splits of the dH GEMM
+// L2 bytes the sweeps' tile walk keeps resident for H: a third of the
+// 126 MB L2, leaving the rest to the streamed W tiles and the G stores.  With
+// a token-tile block wider than this (ragged: 64 tiles x 2 MB of H) every
+// round re-read all of H from HBM (43 GB per sweep instead of 8.5 GB).
+constexpr size_t kL2BudgetSweep = size_t(42) << 20;
 constexpr int kColsumSegs = 8;                  // row segments of the db column sums
 
 using CfgKK = GemmCfg<kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
@@ -146,10 +152,32 @@ struct DynRows {
     int dim = 0;                      // 1: bounds M, 2: bounds K
 };
 
+// Fast-dimension tiles per block of the tile walk: as many as keep one
+// block's panels of the reused operand (panel_bytes each) within `budget`,
+// with the blocks balanced in width.
+int walk_group(int64_t n_fast, size_t panel_bytes, size_t budget) {
+    if (n_fast <= 0) return 1;
+    const int64_t gmax = std::max<int64_t>(1, (int64_t)(budget / std::max<size_t>(panel_bytes, 1)));
+    return (int)cdiv(n_fast, cdiv(n_fast, gmax));
+}
+
+// One block: the walk covers every tile of the fast dimension per step of
+// the slow one.  dH streams both of its operands (K = V); dW's reused H
+// panels measured no gain from blocking (G, the larger operand, is then
+// re-read once per block).
+constexpr int kOneBlock = std::numeric_limits<int>::max();
+
+// How a GEMM's units are walked.
+struct Walk {
+    int n_fastest;        // 1: consecutive tiles share the A panel
+    int k_splits;         // K ranges per tile
+    int group;            // fast-dimension tiles per block of the walk
+};
+
 template <class Cfg, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64_t N, int64_t K,
-                        int n_fastest, int k_splits, const typename Epi::Params& ep, int32_t* err,
-                        int sms, cudaStream_t st, DynRows dyn = DynRows()) {
+                        const Walk& w, const typename Epi::Params& ep, int32_t* err, int sms,
+                        cudaStream_t st, DynRows dyn = DynRows()) {
     GemmGeom g;
     g.dyn_count = dyn.count;
     g.dyn_base = dyn.base;
@@ -158,9 +186,10 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
     g.tiles_m = (int)cdiv(M, Cfg::PAIR_M);
     g.tiles_n = (int)cdiv(N, Cfg::BN);
     g.k_iters = (int)cdiv(K, Cfg::BK);
-    g.k_splits = k_splits;
+    g.k_splits = w.k_splits;
     g.num_tiles = g.tiles_m * g.tiles_n;
-    g.n_fastest = n_fastest;
+    g.n_fastest = w.n_fastest;
+    g.group = w.group;
     if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
     auto kern = umma_gemm_kernel<Cfg, Epi>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -483,6 +512,11 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
         lp.v0 = h->v0;
 
         CUtensorMap mH_k, mH_mn, mG_k, mG_mn;
+        // the sweeps walk vocabulary tiles under a block of token tiles
+        // whose H panels stay in L2 (H is re-read from L2, not HBM)
+        const Walk sweep_walk{0, 1,
+                              walk_group(cdiv(rows, CfgKK::PAIR_M),
+                                         (size_t)CfgKK::PAIR_M * D * 2, kL2BudgetSweep)};
         if (bf16) {
             const void* Hc = static_cast<const __nv_bfloat16*>(H) + r0 * D;
             if (!make_map(&mH_k, Hc, D, rows, D, 64, 128)) return FLDCE_ERR_CUDA;
@@ -490,7 +524,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
         // sweep 1 (not needed when every shard's statistics are given)
         if (mode != MERGE_GATHERED) {
             if (bf16) {
-                FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, 0, 1, lp,
+                FLDCE_CUDA((launch_gemm<CfgKK, LseEpi>(mH_k, mW_k, rows, V, D, sweep_walk, lp,
                                                        &cnt->dev_err, dev.sms, st,
                                                        DynRows{dynp, (int)r0, 1})));
             } else {
@@ -567,8 +601,9 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             gp.eps_over_V = eps / (float)h->Vtot;
             gp.one_minus_eps = 1.f - eps;
             gp.bias = static_cast<const __nv_bfloat16*>(bias);
-            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, 0, 1, gp, &cnt->dev_err,
-                                                 dev.sms, st, DynRows{dynp, (int)r0, 1})));
+            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, sweep_walk, gp,
+                                                 &cnt->dev_err, dev.sms, st,
+                                                 DynRows{dynp, (int)r0, 1})));
             prof_mark(h, PK_G, st);
             if (bias != nullptr) {
                 FLDCE_CUDA(launch_colsum(G, true, h->Vpad, rows, V, db_part, db_acc, ci > 0, st,
@@ -606,7 +641,8 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
                     if (!make_store_map(&hp.omap, dHc, D, rows, D, 2)) return FLDCE_ERR_CUDA;
                     hp.mode = OUT_BF16;
                 }
-                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, 1, ks, hp,
+                const Walk dh_walk{1, ks, kOneBlock};
+                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, dh_walk, hp,
                                                          &cnt->dev_err, dev.sms, st,
                                                          DynRows{dynp, (int)r0, 1})));
                 prof_mark(h, PK_DH, st);
@@ -628,8 +664,9 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
                     if (!make_store_map(&wp.omap, dw_ws, D, V, D, 4)) return FLDCE_ERR_CUDA;
                     wp.mode = ci == 0 ? WS_STORE : WS_ADD;
                 }
-                FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, 1, 1, wp,
-                                                         &cnt->dev_err, dev.sms, st,
+                const Walk dw_walk{1, 1, kOneBlock};
+                FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, dw_walk,
+                                                         wp, &cnt->dev_err, dev.sms, st,
                                                          DynRows{dynp, (int)r0, 2})));
                 prof_mark(h, PK_DW, st);
                 if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {

@@ -73,6 +73,11 @@ struct GemmGeom {
     int k_splits;         // K ranges per tile (1 to 4)
     int num_tiles;        // tiles_m * tiles_n
     int n_fastest;        // 1: consecutive tiles walk n first (share the A panel)
+    // The walk covers the fast dimension in blocks of `group` tiles: all
+    // tiles of one block along the slow dimension, then the next block.  The
+    // operand panels of one block stay in L2 while the other operand
+    // streams past them; group >= the fast dimension's tiles is one block.
+    int group;
     // Optional row count known only on the device (compacted tokens): the
     // live rows are clamp(*dyn_count - dyn_base, 0, dyn_cap), bounding M
     // (dyn_dim == 1) or K (dyn_dim == 2).  The host sizes the launch for
@@ -225,15 +230,23 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         *abort_flag = 1;
         if (lane == 0) atomicOr(err, FLDCE_DEV_ERR_TIMEOUT);
     };
+    const int n_fast = geom.n_fastest ? geom.tiles_n : geom.tiles_m;
+    const int n_slow = geom.n_fastest ? geom.tiles_m : geom.tiles_n;
+    const int grp = max(1, min(geom.group, n_fast));
     auto unit_coords = [&](int u, int& mt, int& nt, int& split, int& k0, int& k1) {
         split = u / geom.num_tiles;
         const int tile = u - split * geom.num_tiles;
+        const int blk = tile / (grp * n_slow);
+        const int r = tile - blk * (grp * n_slow);
+        const int f0 = blk * grp;
+        const int gb = min(grp, n_fast - f0);          // the last block may be narrower
+        const int f = f0 + r % gb, sl = r / gb;
         if (geom.n_fastest) {
-            nt = tile % geom.tiles_n;
-            mt = tile / geom.tiles_n;
+            nt = f;
+            mt = sl;
         } else {
-            mt = tile % geom.tiles_m;
-            nt = tile / geom.tiles_m;
+            mt = f;
+            nt = sl;
         }
         k0 = split * kps;
         k1 = min(geom.k_iters, k0 + kps);
@@ -241,6 +254,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
+        // evict_first on the streamed operand / evict_last on the reused one
+        // measured more HBM traffic than the default priority, not less
         const uint64_t pol = l2_policy_evict_normal();
         const uint32_t lead_full0 = mapa_shared(full_bar(0), 0);
         uint32_t it = 0;

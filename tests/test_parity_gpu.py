@@ -212,3 +212,13 @@ def test_split_dh(V, dh_fp32):
     _full_compare(wl, g, "bf16")
     g2 = run_gpu(wl, plan=g["plan"])
     assert torch.equal(g["dH"], g2["dH"])
+
+
+# With D = 4096 each 256-token tile of H is 2 MB; 22 token tiles (5500 tokens,
+# the last tile ragged) exceed the sweeps' L2 block, so the sweeps walk the
+# vocabulary under two blocks of 11 token tiles.  Every tile is still visited
+# exactly once.
+def test_sweeps_walk_token_tiles_in_l2_blocks():
+    wl = _small(5500, 4096, 1500, seed=15, label_smoothing=0.1)
+    g = run_gpu(wl)
+    _full_compare(wl, g, "bf16")
