@@ -67,6 +67,14 @@ extern "C" {
 /* dH is written as fp32 instead of the dtype (e.g. partial dH summed over
  * vocabulary shards).  Not with FLDCE_FLAG_SKIP_IGNORED. */
 #define FLDCE_FLAG_DH_FP32       0x4u
+/* dW (and db) are accumulated into: dW += G^T H, db += sum_n G[n, :], for
+ * gradient accumulation over micro-batches.  The caller initialises them
+ * (e.g. to zero) before the first call.  A bf16 dW gets the call's fp32
+ * gradient added and is rounded once; an fp32 dW (FLDCE_FLAG_DW_FP32 or the
+ * fp32 dtype) takes the chunks' fp32 reduce-adds directly.  N == 0 leaves dW
+ * and db as they are.  dH is still overwritten.  The pages always overwrite
+ * (their dW is a fresh buffer per call); this flag is an extension. */
+#define FLDCE_FLAG_DW_ACCUMULATE 0x8u
 
 typedef struct fldce_plan* fldce_handle;
 
@@ -108,7 +116,7 @@ int fldce_workspace_size(fldce_handle h, int64_t N, size_t* bytes);
 
 /*
  * fldce_chunk_size -- tokens per internal chunk the plan uses (the explicit
- * chunk_N, or the library's choice: the largest multiple of 128 tokens whose
+ * chunk_N, or the library's choice: the largest multiple of 256 tokens whose
  * G buffer stays within 4 GiB, capped at max_N).
  * Errors: INVALID_ARG (null handle or out).
  */
@@ -124,7 +132,8 @@ int fldce_chunk_size(fldce_handle h, int64_t* chunk_N);
  *   W        [device, in]  [V, D] dtype.
  *   target   [device, in]  [N] int64.
  *   p_mask   [device, in]  [N] fp32, or NULL for p = 1 (ordinary CE).
- *   N        tokens, 0 <= N <= max_N.  N == 0 writes loss = 0 and dW = 0.
+ *   N        tokens, 0 <= N <= max_N.  N == 0 writes loss = 0 and dW = 0
+ *            (leaves dW as it is with FLDCE_FLAG_DW_ACCUMULATE).
  *   total    T > 0 is used as given ('mean' over an explicit normaliser;
  *            'sum' is T = 1); T <= 0 means the count of non-ignored,
  *            in-range targets, computed on the device (no host sync).
@@ -137,7 +146,7 @@ int fldce_chunk_size(fldce_handle h, int64_t* chunk_N);
  *                   z[n,v] = max_v z[n,v] (every row).
  *   dH       [device, out] [N, D] dtype; overwritten.
  *   dW       [device, out] [V, D] dtype (fp32 with FLDCE_FLAG_DW_FP32);
- *            overwritten (not accumulated into).
+ *            overwritten, or added to with FLDCE_FLAG_DW_ACCUMULATE.
  *   workspace        [device] scratch of at least fldce_workspace_size(N)
  *                    bytes, 256-byte aligned; contents need no initialisation
  *                    and are undefined afterwards.  Calls that share a
@@ -205,7 +214,8 @@ int fldce_fwd_bwd_noalloc(fldce_handle h,
  *             (the page's F.linear(x, weight, bias) before the scale).
  *   db        [device, out] [V] dtype (fp32 with FLDCE_FLAG_DW_FP32);
  *             required when bias is set: db[v] = sum_n G[n, v] (the page's
- *             db += dlogits.sum(0)), summed in a fixed order.
+ *             db += dlogits.sum(0)), summed in a fixed order (added to
+ *             db with FLDCE_FLAG_DW_ACCUMULATE).
  *   count_dev [device, in, may be NULL] 1 int32: when total <= 0, the
  *             normaliser is *count_dev instead of this call's own count --
  *             e.g. the job-wide count of valid tokens, summed over

@@ -32,6 +32,7 @@ FLDCE_FP32 = 1
 FLDCE_FLAG_DW_FP32 = 0x1
 FLDCE_FLAG_SKIP_IGNORED = 0x2
 FLDCE_FLAG_DH_FP32 = 0x4
+FLDCE_FLAG_DW_ACCUMULATE = 0x8
 
 # every symbol include/fldce.h declares
 EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
@@ -318,7 +319,7 @@ class Plan:
                  chunk_N: int = 0, logit_scale: float = 1.0, label_smoothing: float = 0.0,
                  ignore_index: int = -100, dw_fp32: bool = False, skip_ignored: bool = False,
                  dh_fp32: bool = False, vocab_start: int = 0, vocab_total: int = 0,
-                 device=None):
+                 dw_accumulate: bool = False, device=None):
         code = FLDCE_BF16 if dtype == torch.bfloat16 else FLDCE_FP32
         if _TORCH_DTYPE[code] != dtype:
             raise TypeError(f"unsupported dtype {dtype}")
@@ -332,9 +333,11 @@ class Plan:
             label_smoothing=label_smoothing, ignore_index=ignore_index,
             flags=(FLDCE_FLAG_DW_FP32 if dw_fp32 else 0) |
             (FLDCE_FLAG_SKIP_IGNORED if skip_ignored else 0) |
-            (FLDCE_FLAG_DH_FP32 if dh_fp32 else 0),
+            (FLDCE_FLAG_DH_FP32 if dh_fp32 else 0) |
+            (FLDCE_FLAG_DW_ACCUMULATE if dw_accumulate else 0),
             vocab_start=vocab_start, vocab_total=vocab_total)
         self.dh_fp32 = bool(dh_fp32)
+        self.dw_accumulate = bool(dw_accumulate)
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
 
     def close(self):
@@ -349,13 +352,16 @@ class Plan:
             pass
 
     def outputs(self, N: int, *, want_rows: bool = True, want_argmax: bool = False):
+        """Output buffers for N tokens; dW starts at zero for a plan that
+        accumulates into it."""
         dev = self.device
+        new_dw = torch.zeros if self.dw_accumulate else torch.empty
         out = {
             "loss": torch.empty(1, dtype=torch.float32, device=dev),
             "dH": torch.empty(N, self.D, dtype=torch.float32 if self.dh_fp32 else self.dtype,
                               device=dev),
-            "dW": torch.empty(self.V, self.D,
-                              dtype=torch.float32 if self.dw_fp32 else self.dtype, device=dev),
+            "dW": new_dw(self.V, self.D,
+                         dtype=torch.float32 if self.dw_fp32 else self.dtype, device=dev),
             "err": torch.empty(2, dtype=torch.int32, device=dev),
         }
         if want_rows:
@@ -372,8 +378,9 @@ class Plan:
         if out is None:
             out = self.outputs(N, **kw)
             if bias is not None:
-                out["db"] = torch.empty(self.V, device=self.device,
-                                        dtype=torch.float32 if self.dw_fp32 else self.dtype)
+                new_db = torch.zeros if self.dw_accumulate else torch.empty
+                out["db"] = new_db(self.V, device=self.device,
+                                   dtype=torch.float32 if self.dw_fp32 else self.dtype)
         if bias is None and count_dev is None and dw_ready_event is None:
             fldce_fwd_bwd(self.handle, H, W, target, p_mask, N, total, grad_out, out["loss"],
                           out.get("loss_per_token"), out.get("lse"), out.get("argmax"),

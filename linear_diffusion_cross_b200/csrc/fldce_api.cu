@@ -232,11 +232,13 @@ cudaError_t launch_sum_splits(const float* part, int64_t stride, int k, void* ds
     return cudaGetLastError();
 }
 
-cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, int sms, cudaStream_t st) {
+// dst = bf16(src), or bf16(dst + src) with add.
+cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, bool add, int sms,
+                           cudaStream_t st) {
     const int64_t n8 = n / 8;
     if (n8 == 0) return cudaSuccess;
     const int blocks = (int)std::min<int64_t>(cdiv(n8, 256), 8 * (int64_t)sms);
-    k_f32_to_bf16<<<blocks, 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), n8);
+    k_f32_to_bf16<<<blocks, 256, 0, st>>>(src, static_cast<__nv_bfloat16*>(dst), n8, add ? 1 : 0);
     return cudaGetLastError();
 }
 
@@ -298,6 +300,8 @@ bool dw_out_fp32(const fldce_plan* p) {
     return p->cfg.dtype == FLDCE_FP32 || (p->cfg.flags & FLDCE_FLAG_DW_FP32) != 0;
 }
 
+bool dw_accumulate(const fldce_plan* p) { return (p->cfg.flags & FLDCE_FLAG_DW_ACCUMULATE) != 0; }
+
 Layout make_layout(const fldce_plan* p, int64_t N) {
     Layout L{};
     const int64_t C = std::max<int64_t>(1, std::min<int64_t>(p->chunk, N));
@@ -324,7 +328,8 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
     L.dh_acc = take(p->cfg.dtype == FLDCE_BF16
                         ? (size_t)kMaxKSplits * round_up((size_t)C, 256) * p->cfg.D * 4
                         : 0);
-    const bool acc = L.nchunks > 1 && !dw_out_fp32(p);
+    // fp32 dW partials across chunks, or before adding into a bf16 dW
+    const bool acc = (L.nchunks > 1 || (dw_accumulate(p) && N > 0)) && !dw_out_fp32(p);
     L.dw_acc = take(acc ? (size_t)p->cfg.V * p->cfg.D * 4 : 0);
     L.db_part = take((size_t)kColsumSegs * p->cfg.V * 4);
     L.db_acc = take((size_t)p->cfg.V * 4);
@@ -414,6 +419,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
                                               : reinterpret_cast<float*>(ws + L.loss_tok);
     const bool bf16 = cfg.dtype == FLDCE_BF16;
     const bool skip = (cfg.flags & FLDCE_FLAG_SKIP_IGNORED) != 0;
+    const bool accum = dw_accumulate(h);     // dW (and db) += this call's gradient
     // compaction buffers (FLDCE_FLAG_SKIP_IGNORED) and the caller's outputs
     int32_t* c_idx = reinterpret_cast<int32_t*>(ws + L.c_idx);
     int32_t* c_pos = reinterpret_cast<int32_t*>(ws + L.c_pos);
@@ -465,7 +471,7 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             if (backward) dH = c_dH;
             dynp = &cnt->n_compact;
         }
-    } else if (backward) {
+    } else if (backward && !accum) {
         FLDCE_CUDA(cudaMemsetAsync(dW, 0, (size_t)V * D * (dw_out_fp32(h) ? 4 : h->elt), st));
         if (bias != nullptr)
             FLDCE_CUDA(cudaMemsetAsync(db, 0, (size_t)V * (dw_out_fp32(h) ? 4 : h->elt), st));
@@ -474,10 +480,11 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
     const bool fp32_dw = dw_out_fp32(h);
     float* dw_ws = fp32_dw ? static_cast<float*>(dW) : reinterpret_cast<float*>(ws + L.dw_acc);
 
-    if (skip && backward && N > 0) {
+    if (skip && backward && N > 0 && !(accum && fp32_dw)) {
         // with no token to carry a loss the dW GEMM has no K rows: zero the
-        // buffer its first chunk would have written
-        const bool direct = L.nchunks == 1 && !fp32_dw;
+        // buffer its first chunk would have written (an fp32 dW accumulated
+        // into is left as it is)
+        const bool direct = L.nchunks == 1 && !fp32_dw && !accum;
         void* dst = direct ? dW : static_cast<void*>(dw_ws);
         const int64_t b16 = (int64_t)V * D * (direct ? 2 : 4) / 16;
         k_zero_if_none<<<(unsigned)std::min<int64_t>(cdiv(b16, 256), 8 * (int64_t)dev.sms), 256, 0,
@@ -577,13 +584,14 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
 
         // dW: one chunk writes the output directly; several chunks store, then
         // reduce-add, fp32 partial sums (into dW itself when it is fp32).
-        const int simt_mode = L.nchunks == 1 ? 0 : (ci == 0 ? 1 : 2);
+        const int simt_mode = accum ? 2 : (L.nchunks == 1 ? 0 : (ci == 0 ? 1 : 2));
         const bool dw_first = call.dw_ready_event != nullptr && ci + 1 == L.nchunks;
         // db is final once the last chunk's column sums are in: cast it out
         auto finish_db = [&]() -> int {
             if (bias == nullptr || ci + 1 != L.nchunks) return FLDCE_OK;
             k_cast_out<<<(unsigned)cdiv(V, 256), 256, 0, st>>>(db_acc, db, V,
-                                                              dw_out_fp32(h) ? 0 : 1);
+                                                              dw_out_fp32(h) ? 0 : 1,
+                                                              accum ? 1 : 0);
             FLDCE_CUDA(cudaGetLastError());
             prof_mark(h, PK_DB, st);
             return FLDCE_OK;
@@ -657,20 +665,22 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             // directly; several store, then reduce-add, fp32 partial sums.
             auto do_dw = [&]() -> int {
                 StoreEpi::Params wp;
-                if (L.nchunks == 1 && !fp32_dw) {
+                if (L.nchunks == 1 && !fp32_dw && !accum) {
                     if (!make_store_map(&wp.omap, dW, D, V, D, 2)) return FLDCE_ERR_CUDA;
                     wp.mode = OUT_BF16;
                 } else {
+                    // fp32 partial sums; an fp32 dW accumulated into takes
+                    // every chunk's reduce-add directly
                     if (!make_store_map(&wp.omap, dw_ws, D, V, D, 4)) return FLDCE_ERR_CUDA;
-                    wp.mode = ci == 0 ? WS_STORE : WS_ADD;
+                    wp.mode = (ci == 0 && !(accum && fp32_dw)) ? WS_STORE : WS_ADD;
                 }
                 const Walk dw_walk{1, 1, kOneBlock};
                 FLDCE_CUDA((launch_gemm<CfgMM, StoreEpi>(mG_mn, mH_mn, (int)V, D, rows, dw_walk,
                                                          wp, &cnt->dev_err, dev.sms, st,
                                                          DynRows{dynp, (int)r0, 2})));
                 prof_mark(h, PK_DW, st);
-                if (L.nchunks > 1 && !fp32_dw && ci + 1 == L.nchunks) {
-                    FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, dev.sms, st));
+                if ((L.nchunks > 1 || accum) && !fp32_dw && ci + 1 == L.nchunks) {
+                    FLDCE_CUDA(launch_to_bf16(dw_ws, dW, V * D, accum, dev.sms, st));
                     prof_mark(h, PK_CONVERT, st);
                 }
                 return FLDCE_OK;
@@ -744,7 +754,8 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
         return FLDCE_ERR_INVALID_ARG;
     if (!std::isfinite(cfg->logit_scale) || cfg->logit_scale == 0.f) return FLDCE_ERR_INVALID_ARG;
     if (cfg->dtype != FLDCE_BF16 && cfg->dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
-    if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED | FLDCE_FLAG_DH_FP32)) != 0)
+    if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED | FLDCE_FLAG_DH_FP32 |
+                        FLDCE_FLAG_DW_ACCUMULATE)) != 0)
         return FLDCE_ERR_UNSUPPORTED;
     if ((cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0 &&
         (cfg->dtype != FLDCE_BF16 || (cfg->flags & FLDCE_FLAG_DH_FP32) != 0))

@@ -652,13 +652,23 @@ __global__ void k_finish(const float* __restrict__ loss_tok, int64_t N, const Co
     }
 }
 
-// fp32 -> bf16 (round to nearest even), 8 elements per thread and step.
+// fp32 -> bf16 (round to nearest even), 8 elements per thread and step;
+// with add, dst = bf16(dst + src) (an accumulated gradient, rounded once).
 __global__ void k_f32_to_bf16(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
-                              int64_t n8) {
+                              int64_t n8, int add) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const float4 a = reinterpret_cast<const float4*>(src)[2 * i];
-        const float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+        float4 a = reinterpret_cast<const float4*>(src)[2 * i];
+        float4 b = reinterpret_cast<const float4*>(src)[2 * i + 1];
+        if (add) {
+            const uint4 o = reinterpret_cast<const uint4*>(dst)[i];
+            const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+            const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+            const float2 o2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.z));
+            const float2 o3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.w));
+            a.x += o0.x; a.y += o0.y; a.z += o1.x; a.w += o1.y;
+            b.x += o2.x; b.y += o2.y; b.z += o3.x; b.w += o3.y;
+        }
         uint4 w;
         w.x = pack_bf16x2(a.x, a.y);
         w.y = pack_bf16x2(a.z, a.w);
@@ -787,12 +797,19 @@ __global__ void k_colsum_final(const float* __restrict__ part, int nseg, int64_t
     acc[v] = add ? acc[v] + s : s;
 }
 
-// fp32 -> bf16 or fp32 copy, one element per thread (short vectors, any n).
-__global__ void k_cast_out(const float* __restrict__ src, void* dst, int64_t n, int to_bf16) {
+// fp32 -> bf16 or fp32 copy, one element per thread (short vectors, any n);
+// with add, dst += src (rounded once to the output type).
+__global__ void k_cast_out(const float* __restrict__ src, void* dst, int64_t n, int to_bf16,
+                           int add) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
-    if (to_bf16) static_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(src[i]);
-    else static_cast<float*>(dst)[i] = src[i];
+    if (to_bf16) {
+        __nv_bfloat16* d = static_cast<__nv_bfloat16*>(dst);
+        d[i] = __float2bfloat16_rn(add ? src[i] + __bfloat162float(d[i]) : src[i]);
+    } else {
+        float* d = static_cast<float*>(dst);
+        d[i] = add ? src[i] + d[i] : src[i];
+    }
 }
 
 // ======================================================================

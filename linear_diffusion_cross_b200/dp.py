@@ -70,7 +70,12 @@ def fwd_bwd_data_parallel(kernels, H, W, target, p_mask, *, total: float = 0.0,
                           group=None) -> dict:
     """One data-parallel step.  H, target, p_mask: this rank's tokens; W, bias:
     replicated.  ``total > 0`` must already be the job-wide normaliser.
-    Returns this rank's outputs with dW, db and loss summed over ranks."""
+    Returns this rank's outputs with dW, db and loss summed over ranks.
+    A plan that accumulates dW is refused: each step's sum over ranks would
+    add the earlier steps' gradients once per rank."""
+    plan = getattr(kernels, "plan", None)
+    if plan is not None and getattr(plan, "dw_accumulate", False):
+        raise ValueError("fwd_bwd_data_parallel needs a plan that overwrites dW")
     count = None
     if total <= 0:
         count = kernels.count_valid(target)

@@ -94,7 +94,7 @@ def test_workspace_and_chunking(lib):
     h, ws = B.fldce_create(B.FLDCE_BF16, 4096, 256000, 32768)
     try:
         c = B.fldce_chunk_size(h)
-        assert c % 128 == 0 and c * 256000 * 2 <= 1 << 32 and c < 32768
+        assert c % 256 == 0 and c * 256000 * 2 <= 1 << 32 and c < 32768
         # chunked: G for one chunk plus the fp32 dW accumulator
         assert ws >= c * 256000 * 2 + 256000 * 4096 * 4
     finally:
@@ -109,6 +109,21 @@ def test_workspace_and_chunking(lib):
         assert B.fldce_chunk_size(h) == 16
     finally:
         B.fldce_destroy(h)
+
+
+def test_accumulate_workspace(lib):
+    # a bf16 dW accumulated into needs the fp32 accumulator even in one chunk;
+    # an fp32 dW takes the reduce-adds directly and needs none
+    D, V, N = 2560, 151936, 8192
+    sizes = {}
+    for name, flags in [("plain", 0), ("acc", B.FLDCE_FLAG_DW_ACCUMULATE),
+                        ("fp32", B.FLDCE_FLAG_DW_FP32),
+                        ("fp32_acc", B.FLDCE_FLAG_DW_FP32 | B.FLDCE_FLAG_DW_ACCUMULATE)]:
+        h, ws = B.fldce_create(B.FLDCE_BF16, D, V, N, flags=flags)
+        B.fldce_destroy(h)
+        sizes[name] = ws
+    assert sizes["acc"] >= sizes["plain"] + V * D * 4
+    assert sizes["fp32_acc"] == sizes["fp32"] == sizes["plain"]
 
 
 def test_profile_kinds(lib):

@@ -103,3 +103,15 @@ def test_data_parallel_exchange_matches_whole_batch(total, use_bias):
             assert np.allclose(r["dH"], ref.dH[sl], rtol=1e-11, atol=1e-15)
             if use_bias:
                 assert np.allclose(r["db"], ref.db, rtol=1e-11, atol=1e-15)
+
+
+def test_accumulating_plan_is_refused():
+    """Summing an accumulated dW over ranks every step would add the earlier
+    steps once per rank: the data-parallel step refuses such a plan before
+    any collective."""
+    from types import SimpleNamespace
+
+    from linear_diffusion_cross_b200.dp import fwd_bwd_data_parallel
+    kernels = SimpleNamespace(plan=SimpleNamespace(dw_accumulate=True))
+    with pytest.raises(ValueError):
+        fwd_bwd_data_parallel(kernels, None, None, None, None, total=1.0)

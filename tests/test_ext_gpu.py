@@ -121,3 +121,49 @@ def test_scale_in_place(dtype, n):
     B.fldce_scale(x, n, B.FLDCE_BF16 if dtype == torch.bfloat16 else B.FLDCE_FP32, one)
     torch.cuda.synchronize()
     assert torch.equal(x, (x0.float() * 2.5).to(dtype))
+
+
+# FLDCE_FLAG_DW_ACCUMULATE: two micro-batches with the same weight, dW and db
+# accumulated over both, dH and the loss of the second call alone.
+@pytest.mark.parametrize("D,V,chunk,dw_fp32,dtype,skip", [
+    (136, 1003, 0, False, torch.bfloat16, False),     # one chunk: fp32 partial, then added
+    (136, 1003, 128, False, torch.bfloat16, False),   # several chunks
+    (64, 2049, 100, True, torch.bfloat16, False),     # fp32 dW takes the reduce-adds
+    (64, 257, 32, False, torch.float32, False),       # CUDA-core path
+    (136, 1003, 0, False, torch.bfloat16, True),      # compacted tokens
+], ids=["bf16_1chunk", "bf16_chunks", "dw_fp32", "fp32", "skip"])
+def test_dw_accumulate(D, V, chunk, dw_fp32, dtype, skip):
+    w1 = _wl(300, D, V, seed=21, dtype=dtype, label_smoothing=0.1, grad_out=1.25)
+    w2 = _wl(257, D, V, seed=22, dtype=dtype, label_smoothing=0.1, grad_out=1.25)
+    w2.W = w1.W
+    b = _bias(V, dtype, 3)
+    plan = B.Plan(D, V, 300, dtype=dtype, chunk_N=chunk, label_smoothing=0.1, dw_fp32=dw_fp32,
+                  skip_ignored=skip, dw_accumulate=True, device=DEV)
+    out = plan.outputs(300)
+    out["db"] = torch.zeros(V, device=DEV, dtype=torch.float32 if dw_fp32 else dtype)
+    assert torch.count_nonzero(out["dW"]) == 0
+    Wd, bd = w1.W.to(DEV), b.to(DEV)
+    for wl in (w1, w2):
+        o = {k: (v[:wl.N] if k in ("dH", "loss_per_token", "lse") else v) for k, v in out.items()}
+        plan.fwd_bwd(wl.H.to(DEV), Wd, wl.target.to(DEV), wl.p_mask.to(DEV), wl.total,
+                     wl.grad_out, out=o, bias=bd)
+    torch.cuda.synchronize()
+    r1, r2 = _oracle(w1, b), _oracle(w2, b)
+    key = "bf16" if dtype == torch.bfloat16 else "fp32"
+    assert maxabs_err(f64(out["dW"]), r1.dW + r2.dW) <= GRAD_TOL[key]
+    assert maxabs_err(f64(out["db"]), r1.db + r2.db) <= GRAD_TOL[key]
+    assert maxabs_err(f64(out["dH"][:w2.N]), r2.dH) <= GRAD_TOL[key]
+    assert abs(float(out["loss"][0]) - r2.loss) <= LOSS_RTOL * abs(r2.loss)
+    # a call with no tokens, and one whose tokens are all ignored, add nothing
+    before = (out["dW"].clone(), out["db"].clone())
+    empty = torch.empty(0, D, dtype=dtype, device=DEV)
+    o0 = dict(out, dH=out["dH"][:0], loss_per_token=out["loss_per_token"][:0],
+              lse=out["lse"][:0])
+    plan.fwd_bwd(empty, Wd, torch.empty(0, dtype=torch.int64, device=DEV), None, 1.0,
+                 out=o0, bias=bd)
+    ign = torch.full((64,), -100, dtype=torch.int64, device=DEV)
+    o1 = dict(out, dH=out["dH"][:64], loss_per_token=out["loss_per_token"][:64],
+              lse=out["lse"][:64])
+    plan.fwd_bwd(w1.H[:64].to(DEV), Wd, ign, None, 0.0, out=o1, bias=bd)
+    torch.cuda.synchronize()
+    assert torch.equal(out["dW"], before[0]) and torch.equal(out["db"], before[1])
