@@ -74,6 +74,8 @@ class HostPipeline:
         losses = torch.empty(len(batches), dtype=torch.float32).pin_memory()
         if not batches:
             return losses
+        # no copy starts before the work already queued on the compute stream
+        self.copy_stream.wait_stream(stream)
         self._fill(0, batches[0])
         for i in range(len(batches)):
             if i + 1 < len(batches):
