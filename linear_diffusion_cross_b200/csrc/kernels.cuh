@@ -21,6 +21,37 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Two fp32 lanes per instruction (sm_100 f32x2 arithmetic), each rounded to
+// nearest exactly as the scalar operation would be.
+__device__ __forceinline__ void mul2(float& x, float& y, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(x), "=f"(y) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void add2(float& x, float& y, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(x), "=f"(y) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void fma2(float& x, float& y, float a0, float a1, float b0, float b1,
+                                     float c0, float c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(x), "=f"(y) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -121,7 +152,8 @@ struct LseEpi {
             }
             float tv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) tv[i] = __uint_as_float(r[i]) * p.c;
+            for (int i = 0; i < 32; i += 2)
+                mul2(tv[i], tv[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.c, p.c);
             if (32 * j + 32 > ncols) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
@@ -130,10 +162,10 @@ struct LseEpi {
             float cm0 = fmaxf(tv[0], tv[1]), cm1 = fmaxf(tv[2], tv[3]);
 #pragma unroll
             for (int i = 4; i < 32; i += 4) {
-                cm0 = fmaxf(cm0, fmaxf(tv[i], tv[i + 1]));
-                cm1 = fmaxf(cm1, fmaxf(tv[i + 2], tv[i + 3]));
+                cm0 = fmax3(cm0, tv[i], tv[i + 1]);
+                cm1 = fmax3(cm1, tv[i + 2], tv[i + 3]);
             }
-            const float nm = fmaxf(mx, fmaxf(cm0, cm1));
+            const float nm = fmax3(mx, cm0, cm1);
             if (want_am) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
@@ -156,10 +188,11 @@ struct LseEpi {
             float e0 = 0.f, e1 = 0.f, e2 = 0.f, e3 = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-                e0 += ex2(tv[i] - nm);
-                e1 += ex2(tv[i + 1] - nm);
-                e2 += ex2(tv[i + 2] - nm);
-                e3 += ex2(tv[i + 3] - nm);
+                float d0, d1, d2, d3;
+                add2(d0, d1, tv[i], tv[i + 1], -nm, -nm);
+                add2(d2, d3, tv[i + 2], tv[i + 3], -nm, -nm);
+                add2(e0, e1, e0, e1, ex2(d0), ex2(d1));
+                add2(e2, e3, e2, e3, ex2(d2), ex2(d3));
             }
             l = l * ex2(mx - nm) + ((e0 + e1) + (e2 + e3));
             mx = nm;
@@ -245,16 +278,24 @@ struct GEpi {
                 float b[32];
                 load_bias32(p.bias, n0 + 32 * j, p.V, b);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    g[i] = fmaf(gc, ex2(fmaf(__uint_as_float(r[i]) + b[i], p.c, -L2)), -base);
+                for (int i = 0; i < 32; i += 2) {
+                    float a0, a1, t0, t1;
+                    add2(a0, a1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), b[i], b[i + 1]);
+                    fma2(t0, t1, a0, a1, p.c, p.c, -L2, -L2);
+                    fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
+                }
                 if (gc == 0.f) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) g[i] = 0.f;
                 }
             } else if (gc != 0.f) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    g[i] = fmaf(gc, ex2(fmaf(__uint_as_float(r[i]), p.c, -L2)), -base);
+                for (int i = 0; i < 32; i += 2) {
+                    float t0, t1;
+                    fma2(t0, t1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.c, p.c, -L2,
+                         -L2);
+                    fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) g[i] = 0.f;
