@@ -53,6 +53,11 @@ constexpr int kColsumSegs = 8;                  // row segments of the db column
 
 using CfgKK = GemmCfg<kStages, false, false>;   // sweeps 1 and 2: H (K-major), W (K-major)
 using CfgKM = GemmCfg<kStages, false, true>;    // dH: G (K-major), W (MN-major)
+// dH with 256 x 512 tiles: two MMAs per staged A tile (48 KB stages, 4 deep).
+// Its K loop runs over the whole vocabulary, so the epilogue that no longer
+// overlaps the MMAs costs little, while the stages per MMA and the operand
+// traffic from L2 drop.
+using CfgKM2 = GemmCfg<4, false, true, 2>;
 using CfgMM = GemmCfg<kStages, true, true>;     // dW: G^T (MN-major), H (MN-major)
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -159,6 +164,35 @@ int walk_group(int64_t n_fast, size_t panel_bytes, size_t budget) {
     if (n_fast <= 0) return 1;
     const int64_t gmax = std::max<int64_t>(1, (int64_t)(budget / std::max<size_t>(panel_bytes, 1)));
     return (int)cdiv(n_fast, cdiv(n_fast, gmax));
+}
+
+// dH's tile width and K splits.  Both widths are costed with the schedule
+// model of choose_k_splits, in units of one 256-column MMA step: a 512-wide
+// unit does twice the MMA work per K step but, with a quarter less operand
+// traffic from L2 and half the pipeline stages per MMA, measured about 4%
+// less time per MMA under the power cap (kWideDhCost).  The wide tiles are
+// not used when they pad D by more than 10% over 256-wide ones.
+constexpr double kWideDhCost = 0.96;
+
+struct DhPlan {
+    bool wide;
+    int k_splits;
+};
+
+DhPlan plan_dh(int64_t rows, int64_t D, int64_t V, int pairs) {
+    const int64_t k_iters = cdiv(V, 64);
+    const int64_t mt = cdiv(rows, 256);
+    auto cost = [&](int64_t tiles, int ks) {
+        return (double)(cdiv(ks * tiles, pairs) * cdiv(k_iters, ks));
+    };
+    const int64_t nt = mt * cdiv(D, 256);
+    const int kn = choose_k_splits(nt, k_iters, pairs);
+    DhPlan p{false, kn};
+    if (round_up((size_t)D, 512) * 10 > round_up((size_t)D, 256) * 11) return p;
+    const int64_t wt = mt * cdiv(D, 512);
+    const int kw = choose_k_splits(wt, k_iters, pairs);
+    if (2.0 * kWideDhCost * cost(wt, kw) < cost(nt, kn)) p = DhPlan{true, kw};
+    return p;
 }
 
 // One block: the walk covers every tile of the fast dimension per step of
@@ -629,9 +663,9 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             // split j stores its fp32 partial in its own buffer and one pass
             // sums them in split order (deterministic) into dH.
             auto do_dh = [&]() -> int {
-                const int64_t dh_tiles = cdiv(rows, CfgKM::PAIR_M) * cdiv(D, CfgKM::BN);
-                const int ks = choose_k_splits(dh_tiles, cdiv(V, CfgKM::BK),
-                                               std::max(1, dev.sms / 2));
+                const DhPlan dp = plan_dh(rows, D, V, std::max(1, dev.sms / 2));
+                const bool wide = dp.wide;
+                const int ks = dp.k_splits;
                 StoreEpi::Params hp;
                 const bool dh_fp32 = (cfg.flags & FLDCE_FLAG_DH_FP32) != 0;
                 float* part = reinterpret_cast<float*>(ws + L.dh_acc);
@@ -650,9 +684,14 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
                     hp.mode = OUT_BF16;
                 }
                 const Walk dh_walk{1, ks, kOneBlock};
-                FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, dh_walk, hp,
-                                                         &cnt->dev_err, dev.sms, st,
-                                                         DynRows{dynp, (int)r0, 1})));
+                if (wide)
+                    FLDCE_CUDA((launch_gemm<CfgKM2, StoreEpi>(mG_k, mW_mn, rows, D, V, dh_walk,
+                                                              hp, &cnt->dev_err, dev.sms, st,
+                                                              DynRows{dynp, (int)r0, 1})));
+                else
+                    FLDCE_CUDA((launch_gemm<CfgKM, StoreEpi>(mG_k, mW_mn, rows, D, V, dh_walk,
+                                                             hp, &cnt->dev_err, dev.sms, st,
+                                                             DynRows{dynp, (int)r0, 1})));
                 prof_mark(h, PK_DH, st);
                 if (ks > 1) {
                     FLDCE_CUDA(launch_sum_splits(part, (int64_t)split_rows * D, ks, dHc,

@@ -81,22 +81,23 @@ __device__ __forceinline__ void load_bias32(const __nv_bfloat16* bias, int64_t c
     }
 }
 
-// Walk the eight 32-column chunks of this thread's accumulator row with the
+// Walk the NCH 32-column chunks of this thread's accumulator row with the
 // next chunk's TMEM load in flight while the current one is processed;
 // `f(r, j)` sees chunk j.  The accumulator is released to the MMA warp as
 // soon as the last chunk has landed in registers.
-template <class F>
+template <int NCH, class F>
 __device__ __forceinline__ void for_each_chunk(const AccRow& acc, F&& f) {
+    static_assert(NCH % 2 == 0, "chunks come in pairs");
     uint32_t ra[32], rb[32];
     acc.load(0, ra);
 #pragma unroll 1
-    for (int j = 0; j < 8; j += 2) {
+    for (int j = 0; j < NCH; j += 2) {
         acc.issue(j + 1, rb);
         f(ra, j);
         acc.wait(rb);
-        if (j + 2 < 8) acc.issue(j + 2, ra); else acc.release();
+        if (j + 2 < NCH) acc.issue(j + 2, ra); else acc.release();
         f(rb, j + 1);
-        if (j + 2 < 8) acc.wait(ra);
+        if (j + 2 < NCH) acc.wait(ra);
     }
 }
 
@@ -139,7 +140,8 @@ struct LseEpi {
         const bool want_am = p.part_am != nullptr, want_sz = p.part_sz != nullptr;
         float mx = -CUDART_INF_F, l = 0.f, sz = 0.f, zyv = 0.f, amv = -CUDART_INF_F;
         int am = 0;
-        for_each_chunk(acc, [&](const uint32_t (&rin)[32], int j) {
+        static_assert(Cfg::NSUB == 1, "one 256-column MMA per vocabulary tile");
+        for_each_chunk<Cfg::NCHUNK>(acc, [&](const uint32_t (&rin)[32], int j) {
             uint32_t r[32];
             if (p.bias != nullptr) {
                 float b[32];
@@ -272,7 +274,8 @@ struct GEpi {
         const float base = gc * p.eps_over_V;
         const float tcorr = gc * p.one_minus_eps;
         const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
-        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
+        static_assert(Cfg::NSUB == 1, "one 256-column MMA per vocabulary tile");
+        for_each_chunk<Cfg::NCHUNK>(acc, [&](const uint32_t (&r)[32], int j) {
             float g[32];
             if (p.bias != nullptr) {
                 float b[32];
@@ -341,7 +344,7 @@ struct StoreEpi {
         const int64_t n0 = t.col0;
         const int y = t.row0 + t.split * p.split_rows + 32 * t.q;
         const int mode = p.mode;
-        for_each_chunk(acc, [&](const uint32_t (&r)[32], int j) {
+        for_each_chunk<Cfg::NCHUNK>(acc, [&](const uint32_t (&r)[32], int j) {
             if (mode == OUT_BF16) {
                 float v[32];
 #pragma unroll

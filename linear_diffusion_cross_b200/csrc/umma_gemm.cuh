@@ -44,25 +44,39 @@ constexpr int kGemmThreads = 192;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s per wait
 constexpr int32_t FLDCE_DEV_ERR_TIMEOUT = 1;
 
-template <int STAGES_, bool A_MN_, bool B_MN_>
+// NSUB_ MMAs of N = 256 per K step make one tile NSUB_ x 256 columns wide.
+// NSUB_ = 1: two 256-column accumulators in TMEM, so the epilogue of one tile
+// overlaps the MMAs of the next.  NSUB_ = 2: one 512-column accumulator (all
+// of TMEM); each A tile in shared memory feeds two MMAs, which halves the
+// pipeline stages per MMA and cuts the L2 -> SM operand traffic by a quarter,
+// at the price of an epilogue that no longer overlaps (worth it only where
+// the K loop is long).
+template <int STAGES_, bool A_MN_, bool B_MN_, int NSUB_ = 1>
 struct GemmCfg {
     static constexpr int BM = 128;                 // accumulator rows per CTA
     static constexpr int PAIR_M = 256;             // rows of a pair tile
-    static constexpr int BN = 256;                 // columns of a tile
-    static constexpr int BN_HALF = 128;            // B rows held per CTA
+    static constexpr int NSUB = NSUB_;
+    static constexpr int MMA_N = 256;              // columns of one MMA
+    static constexpr int BN = MMA_N * NSUB;        // columns of a tile
+    static constexpr int BN_HALF = 128 * NSUB;     // B rows held per CTA
     static constexpr int BK = 64;                  // one 128-byte swizzle span of bf16
     static constexpr int STAGES = STAGES_;
     static constexpr bool A_MN = A_MN_;
     static constexpr bool B_MN = B_MN_;
+    static constexpr int NBUF = NSUB == 1 ? 2 : 1; // accumulators in TMEM
+    static constexpr int NCHUNK = BN / 32;         // 32-column epilogue chunks
     static constexpr uint32_t A_BYTES = BM * BK * 2;
-    static constexpr uint32_t B_BYTES = BN_HALF * BK * 2;
+    static constexpr uint32_t B_BLOCK_BYTES = 128 * BK * 2;   // one MMA's B rows of this CTA
+    static constexpr uint32_t B_BYTES = NSUB * B_BLOCK_BYTES;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
+    static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t EPI_BUF_BYTES = 32 * 128;       // 32 rows x 128 B
     static constexpr uint32_t EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
     static constexpr uint32_t BAR_BYTES = 256;
     static constexpr uint32_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
-    static constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_M, BN, A_MN, B_MN);
+    static constexpr uint32_t IDESC = idesc_bf16_f32(PAIR_M, MMA_N, A_MN, B_MN);
+    static_assert(NSUB == 1 || NSUB == 2, "one or two MMAs per K step");
+    static_assert(NBUF * BN == (int)TMEM_COLS, "accumulators fill TMEM");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -264,7 +278,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int mt, nt, split, k0, k1;
             unit_coords(u, mt, nt, split, k0, k1);
             const int arow = mt * Cfg::PAIR_M + (int)rank * Cfg::BM;
-            const int brow = nt * Cfg::BN + (int)rank * Cfg::BN_HALF;
+            // this CTA's B rows for MMA j: [brow + 256 j, brow + 256 j + 128)
+            const int brow = nt * Cfg::BN + (int)rank * 128;
             for (int k = k0; k < k1; ++k, ++it) {
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1u;
@@ -288,11 +303,15 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     }
                     if (Cfg::B_MN) {
 #pragma unroll
-                        for (int j = 0; j < Cfg::BN_HALF / 64; ++j)
-                            tma_load_2d_pair(sb + j * 8192, &tmB, fb, brow + 64 * j, k * Cfg::BK,
-                                             pol);
+                        for (int i = 0; i < Cfg::BN_HALF / 64; ++i)   // 64-column boxes
+                            tma_load_2d_pair(sb + i * 8192, &tmB, fb,
+                                             brow + Cfg::MMA_N * (i >> 1) + 64 * (i & 1),
+                                             k * Cfg::BK, pol);
                     } else {
-                        tma_load_2d_pair(sb, &tmB, fb, k * Cfg::BK, brow, pol);
+#pragma unroll
+                        for (int j = 0; j < Cfg::NSUB; ++j)          // 128-row boxes
+                            tma_load_2d_pair(sb + j * Cfg::B_BLOCK_BYTES, &tmB, fb, k * Cfg::BK,
+                                             brow + Cfg::MMA_N * j, pol);
                     }
                 }
                 __syncwarp();
@@ -305,8 +324,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             for (int u = pair; u < units && !*abort_flag; u += npairs, ++lt) {
                 int mt, nt, split, k0, k1;
                 unit_coords(u, mt, nt, split, k0, k1);
-                const int b = lt & 1;
-                const uint32_t use = lt >> 1;
+                const int b = Cfg::NBUF == 2 ? (int)(lt & 1u) : 0;
+                const uint32_t use = Cfg::NBUF == 2 ? lt >> 1 : lt;
                 if (!mbar_wait_bounded(tempty_bar(b), (use & 1u) ^ 1u, kWaitLimitNs)) {
                     fail();
                     break;
@@ -331,11 +350,15 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             const uint64_t ad =
                                 Cfg::A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
                                           : smem_desc_sw128(sa + kk * 32, 16, 1024);
-                            const uint64_t bd =
-                                Cfg::B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
-                                          : smem_desc_sw128(sb + kk * 32, 16, 1024);
-                            tc_mma_f16_pair(d_tmem, ad, bd, Cfg::IDESC,
-                                            (k > k0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                            for (int j = 0; j < Cfg::NSUB; ++j) {
+                                const uint32_t bj = sb + (uint32_t)j * Cfg::B_BLOCK_BYTES;
+                                const uint64_t bd =
+                                    Cfg::B_MN ? smem_desc_sw128(bj + kk * 2048, 8192, 1024)
+                                              : smem_desc_sw128(bj + kk * 32, 16, 1024);
+                                tc_mma_f16_pair(d_tmem + (uint32_t)(j * Cfg::MMA_N), ad, bd,
+                                                Cfg::IDESC, (k > k0 || kk > 0) ? 1u : 0u);
+                            }
                         }
                         tc_commit_pair_mc(empty_bar(s), 0x3);
                     }
@@ -356,8 +379,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         for (int u = pair; u < units && !*abort_flag; u += npairs, ++lt) {
             int mt, nt, split, k0, k1;
             unit_coords(u, mt, nt, split, k0, k1);
-            const int b = lt & 1;
-            const uint32_t use = lt >> 1;
+            const int b = Cfg::NBUF == 2 ? (int)(lt & 1u) : 0;
+            const uint32_t use = Cfg::NBUF == 2 ? lt >> 1 : lt;
             if (!mbar_wait_bounded(tfull_bar(b), use & 1u, kWaitLimitNs)) {
                 fail();
                 break;

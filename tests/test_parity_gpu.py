@@ -222,3 +222,16 @@ def test_sweeps_walk_token_tiles_in_l2_blocks():
     wl = _small(5500, 4096, 1500, seed=15, label_smoothing=0.1)
     g = run_gpu(wl)
     _full_compare(wl, g, "bf16")
+
+
+# dH runs on 256 x 512 tiles (two MMAs per staged tile, one 512-column
+# accumulator) when the schedule model prefers them over 256-wide ones: many
+# tiles per pair and D a multiple of 512, or close to one.  These shapes take
+# them: unsplit, in two vocabulary splits (bf16 and fp32 dH), and with D =
+# 1000, whose last tile runs 24 columns past D.
+@pytest.mark.parametrize("N,D,V,dh_fp32", [(4608, 2048, 1000, False), (2304, 2048, 5000, False),
+                                           (2304, 2048, 5000, True), (9472, 1000, 1000, False)])
+def test_wide_dh_tiles(N, D, V, dh_fp32):
+    wl = _small(N, D, V, seed=16, label_smoothing=0.1, grad_out=0.5)
+    g = run_gpu(wl, dh_fp32=dh_fp32)
+    _full_compare(wl, g, "bf16")

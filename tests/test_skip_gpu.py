@@ -78,7 +78,8 @@ def _wl(N, D, V, seed, **kw):
 
 @pytest.mark.parametrize("N,D,V,chunk", [(300, 136, 1003, 0), (513, 64, 2049, 128),
                                          (600, 128, 777, 100), (77, 64, 40, 0),
-                                         (300, 136, 5003, 0), (5500, 4096, 1500, 0)])
+                                         (300, 136, 5003, 0), (5500, 4096, 1500, 0),
+                                         (4608, 2048, 1000, 0)])
 def test_skip_matches_oracle(N, D, V, chunk):
     wl = _wl(N, D, V, N, label_smoothing=0.1, logit_scale=0.7, grad_out=1.3)
     _check(wl, _run(wl, chunk))
