@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -226,9 +227,20 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
     g.group = w.group;
     if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
     auto kern = umma_gemm_kernel<Cfg, Epi>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg::SMEM_BYTES);
+    // The shared-memory opt-in is set once per kernel and device, so calls
+    // after the first make no host-side CUDA calls besides the launch (a
+    // call can then be captured into a CUDA graph).
+    static std::atomic<uint64_t> attr_set{0};
+    int devid = 0;
+    cudaError_t e = cudaGetDevice(&devid);
     if (e != cudaSuccess) return e;
+    const uint64_t bit = devid < 64 ? (uint64_t(1) << devid) : 0;
+    if (bit == 0 || (attr_set.load(std::memory_order_acquire) & bit) == 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit, std::memory_order_release);
+    }
     const int pairs = std::min(g.num_tiles * g.k_splits, std::max(1, sms / 2));
     kern<<<2 * pairs, kGemmThreads, Cfg::SMEM_BYTES, st>>>(a, b, g, ep, err);
     return cudaGetLastError();
