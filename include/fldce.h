@@ -156,7 +156,10 @@ int fldce_chunk_size(fldce_handle h, int64_t* chunk_N);
  *             outside [0, V) that are not ignore_index; [1] = device error
  *             bits, 0 when every kernel completed (1 = a pipeline wait timed
  *             out after 4 s and the results are invalid).
- *   stream    cudaStream_t to enqueue on.
+ *   stream    cudaStream_t to enqueue on.  The call allocates nothing and
+ *             never waits on the host, so it may be captured into a CUDA
+ *             graph; make one call on the device before capturing (the first
+ *             call sets the kernels' shared-memory limits).
  * Errors: INVALID_ARG, ALIGN, WORKSPACE, DEVICE, CUDA (launch failure).
  */
 int fldce_fwd_bwd(fldce_handle h,
