@@ -482,13 +482,42 @@ def traffic_for(kernel: str, workload: str):
         return None
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and blank space, so that an edit of
+    comments alone does not count as a change of the kernels."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":                      # string / char literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def source_hash() -> str:
+    """Hash of the library's device and host code (csrc/, comments ignored):
+    the DRAM traffic of a committed ncu summary is reported only while it
+    matches."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "linear_diffusion_cross_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -54,12 +54,27 @@ def test_traffic_needs_counters_of_the_current_sources():
 def test_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     csrc = tmp_path / "linear_diffusion_cross_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cu").write_text("// v1\n")
+    (csrc / "k.cu").write_text("int v = 1;\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     h = bench.source_hash()
     (tmp_path / "profiles" / "ncu_k_w.txt").write_text(
         f"source_sha256: {h}\ndram_bytes_per_launch: 1.5e9\n")
     assert bench.traffic_for("k", "w") == 1.5e9
-    (csrc / "k.cu").write_text("// v2\n")          # the kernel changed since the capture
+    (csrc / "k.cu").write_text("int v = 2;\n")     # the kernel changed since the capture
     assert bench.traffic_for("k", "w") is None
+
+
+def test_comment_edits_keep_the_source_hash(tmp_path, monkeypatch):
+    csrc = tmp_path / "linear_diffusion_cross_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    f = csrc / "k.cuh"
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f.write_text('// v1\nint a = 1; /* x */ const char* s = "// kept";\n')
+    h1 = bench.source_hash()
+    f.write_text('// v2, reworded\n\nint a = 1;   /* y */ const char* s = "// kept";\n')
+    assert bench.source_hash() == h1
+    f.write_text('int a = 2; const char* s = "// kept";\n')
+    assert bench.source_hash() != h1
+    f.write_text('int a = 1; const char* s = "// changed";\n')
+    assert bench.source_hash() != h1
