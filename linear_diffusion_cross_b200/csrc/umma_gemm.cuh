@@ -3,26 +3,31 @@
 //
 // D[m, n] = sum_k A[m, k] * B[n, k] over bf16 operands with an fp32
 // accumulator in tensor memory (TMEM).  Work is cut into 256 x 256 output
-// tiles (optionally also into K splits).  Each tile belongs to a cluster of
-// two CTAs on neighbouring SMs that issue one tcgen05.mma.cta_group::2 per
-// K step of 16: CTA r of the pair holds rows [128 r, 128 r + 128) of the A
-// tile and of the B tile in its shared memory, and receives rows
-// [128 r, 128 r + 128) of the 256 x 256 accumulator in its TMEM.  Each SM
-// therefore streams 32 KB of operands per 64-wide K step instead of the
-// 48 KB a single-CTA 128 x 256 tile needs, a third less L2 -> SM traffic
-// for the same tensor work.
+// tiles (256 x 512 with GemmCfg NSUB = 2), optionally also into K splits,
+// and walked in a fixed order by a persistent grid of CTA pairs.  Each tile
+// belongs to a cluster of two CTAs on neighbouring SMs that issue
+// tcgen05.mma.cta_group::2 (M = 256, N = 256) per K step of 16: CTA r of the
+// pair holds rows [128 r, 128 r + 128) of the A tile and of each 256-row B
+// block in its shared memory, and receives rows [128 r, 128 r + 128) of the
+// accumulator in its TMEM.  Each SM therefore streams 32 KB of operands per
+// 64-wide K step instead of the 48 KB a single-CTA 128 x 256 tile needs, a
+// third less L2 -> SM traffic for the same tensor work (a quarter less again
+// with NSUB = 2, whose A tile feeds two MMAs).
 //
 // Roles (192 threads per CTA):
 //   warp 0      TMA producer (both CTAs): loads this CTA's halves into a
 //               STAGES-deep ring; completion is counted on the pair leader's
 //               "full" mbarrier, which expects the bytes of both CTAs.
 //   warp 1      MMA issuer (leader CTA only issues; both allocate TMEM):
-//               waits for a full stage, issues four M=256 N=256 K=16 MMAs and
-//               commits the stage back to both producers (multicast commit),
-//               then commits a finished accumulator to both epilogues.
+//               waits for a full stage, issues 4 x NSUB M=256 N=256 K=16 MMAs
+//               and commits the stage back to both producers (multicast
+//               commit), then commits a finished accumulator to both
+//               epilogues.
 //   warps 2..5  epilogue (both CTAs): one accumulator row per thread, read
 //               with tcgen05.ld while the next tile's MMAs run into the other
-//               of the two TMEM accumulators; output tiles leave through a
+//               of the two TMEM accumulators (NSUB = 1; with NSUB = 2 the one
+//               512-column accumulator is drained before the next tile
+//               starts); output tiles leave through a
 //               per-warp 128B-swizzled staging buffer and TMA bulk stores (or
 //               bulk reduce-adds).
 //
