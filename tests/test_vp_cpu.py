@@ -11,7 +11,6 @@ import socket
 import tempfile
 
 import numpy as np
-import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
