@@ -28,6 +28,11 @@
  *   - Layouts are dense row-major.  bf16 is IEEE bfloat16 (stored as
  *     uint16), fp32 is IEEE binary32.  Device pointers of H, W, dH, dW, G
  *     and the workspace must be 16-byte aligned; D must be a multiple of 8.
+ *     target must be 8-byte aligned, and p_mask and the per-token outputs
+ *     (loss_per_token, lse, argmax) 4-byte aligned (their natural
+ *     alignment; FLDCE_ERR_ALIGN otherwise).  Where they are 16-byte aligned
+ *     (as every torch allocation is), the per-token kernels move them as
+ *     128-bit vectors.
  *   - The handle holds host state only (the configuration); it is not
  *     thread-safe: use one handle per host thread, or serialise calls.
  */
@@ -155,7 +160,10 @@ int fldce_chunk_size(fldce_handle h, int64_t* chunk_N);
  *   err_count [device, out, may be NULL] 2 int32: [0] = number of targets
  *             outside [0, V) that are not ignore_index; [1] = device error
  *             bits, 0 when every kernel completed (1 = a pipeline wait timed
- *             out after 4 s and the results are invalid).
+ *             out after 4 s: the results are invalid; the kernel waited,
+ *             bounded again, for the work it had issued before freeing its
+ *             tensor memory, but a caller should treat the CUDA context as
+ *             unreliable after this bit and recreate it).
  *   stream    cudaStream_t to enqueue on.  The call allocates nothing and
  *             never waits on the host, so it may be captured into a CUDA
  *             graph; make one call on the device before capturing (the first

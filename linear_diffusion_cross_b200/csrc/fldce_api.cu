@@ -395,6 +395,7 @@ Layout make_layout(const fldce_plan* p, int64_t N) {
 }
 
 bool aligned16(const void* q) { return (reinterpret_cast<uintptr_t>(q) & 15u) == 0; }
+bool aligned_to(const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; }
 
 int check_device(DeviceInfo* d) {
     if (!device_info(d)) return FLDCE_ERR_CUDA;
@@ -441,6 +442,11 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
         return FLDCE_ERR_WORKSPACE;
     if (!aligned16(H) || !aligned16(W) || (backward && (!aligned16(dH) || !aligned16(dW))))
+        return FLDCE_ERR_ALIGN;
+    // natural alignment of the per-token arrays (the row kernels read and
+    // write them as 128-bit vectors where they are 16-byte aligned)
+    if (!aligned_to(target, 8) || !aligned_to(p_mask, 4) || !aligned_to(loss_tok_out, 4) ||
+        !aligned_to(lse_out, 4) || !aligned_to(argmax_out, 4) || !aligned16(stats_out))
         return FLDCE_ERR_ALIGN;
     const Layout L = make_layout(h, N);
     if (workspace_bytes < L.total) return FLDCE_ERR_WORKSPACE;
@@ -623,6 +629,8 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
         mp.row_lse2 = backward && mode != MERGE_EMIT_STATS ? row_lse2 : nullptr;
         mp.row_gcoef = row_gcoef;
         mp.row_y = row_y;
+        mp.vec = aligned16(mp.target) && aligned16(mp.p_mask) && aligned16(mp.loss_tok) &&
+                 aligned16(mp.lse_out) && aligned16(mp.am_out);
         k_merge_rows<<<(unsigned)cdiv((int64_t)rows * kMergeSub, 256), 256, 0, st>>>(mp);
         FLDCE_CUDA(cudaGetLastError());
         prof_mark(h, PK_MERGE, st);

@@ -373,17 +373,44 @@ struct Counters {
     int32_t n_compact; // compacted tokens (FLDCE_FLAG_SKIP_IGNORED)
 };
 
+// Targets are read two at a time as 16-byte vectors (longlong2).  An int64
+// array is 8-byte aligned, so at most its first element sits before the
+// first 16-byte boundary: that element and an odd last one are read alone.
+struct TargetPairs {
+    const int64_t* head;       // the element before the first boundary, or null
+    const longlong2* pairs;    // 16-byte aligned pairs
+    int64_t n_pairs;
+    const int64_t* tail;       // a last unpaired element, or null
+
+    __device__ __forceinline__ TargetPairs(const int64_t* t, int64_t N) {
+        const int64_t h = (N > 0 && (reinterpret_cast<uintptr_t>(t) & 15u) != 0) ? 1 : 0;
+        head = h ? t : nullptr;
+        pairs = reinterpret_cast<const longlong2*>(t + h);
+        n_pairs = (N - h) / 2;
+        tail = ((N - h) & 1) ? t + N - 1 : nullptr;
+    }
+};
+
 // Count the tokens that carry a loss (the page's target.ne(ignore_index).sum(),
 // without the host round trip) and the malformed targets.
 __global__ void k_count_targets(const int64_t* __restrict__ target, int64_t N, int64_t V,
                                 int64_t ignore_index, Counters* cnt) {
     int valid = 0, bad = 0;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t y = target[i];
+    auto take = [&](int64_t y) {
         if (y != ignore_index) {
             if (y >= 0 && y < V) ++valid; else ++bad;
         }
+    };
+    const TargetPairs tp(target, N);
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (int64_t i = tid; i < tp.n_pairs; i += (int64_t)gridDim.x * blockDim.x) {
+        const longlong2 v = tp.pairs[i];
+        take(v.x);
+        take(v.y);
+    }
+    if (tid == 0) {
+        if (tp.head != nullptr) take(*tp.head);
+        if (tp.tail != nullptr) take(*tp.tail);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -405,13 +432,30 @@ __global__ void k_compact_valid(const int64_t* __restrict__ target, int64_t N, i
                                 int32_t* __restrict__ pos, int32_t* count) {
     __shared__ int warp_tot[32];
     const int T = blockDim.x;
-    const int64_t seg = (N + T - 1) / T;
-    const int64_t a = threadIdx.x * seg;
+    // even segments, so that on a 16-byte aligned array every segment starts
+    // on a pair boundary and is read as longlong2 vectors
+    int64_t seg = (N + T - 1) / T;
+    seg += seg & 1;
+    const bool vec = (reinterpret_cast<uintptr_t>(target) & 15u) == 0;
+    const int64_t a = min(N, threadIdx.x * seg);
     const int64_t b = min(N, a + seg);
+    auto ok = [&](int64_t y) { return y != ignore_index && y >= 0 && y < V; };
+    // the targets of positions i and i + 1 (the second only when i + 1 < b)
+    auto pair_at = [&](int64_t i, int64_t& y0, int64_t& y1) {
+        if (vec && i + 1 < b) {
+            const longlong2 v = *reinterpret_cast<const longlong2*>(target + i);
+            y0 = v.x;
+            y1 = v.y;
+        } else {
+            y0 = target[i];
+            y1 = i + 1 < b ? target[i + 1] : ignore_index;
+        }
+    };
     int c = 0;
-    for (int64_t i = a; i < b; ++i) {
-        const int64_t y = target[i];
-        c += (y != ignore_index && y >= 0 && y < V) ? 1 : 0;
+    for (int64_t i = a; i < b; i += 2) {
+        int64_t y0, y1;
+        pair_at(i, y0, y1);
+        c += (ok(y0) ? 1 : 0) + (i + 1 < b && ok(y1) ? 1 : 0);
     }
     // exclusive scan of c over the block
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -434,13 +478,16 @@ __global__ void k_compact_valid(const int64_t* __restrict__ target, int64_t N, i
     }
     __syncthreads();
     int off = incl - c + (w > 0 ? warp_tot[w - 1] : 0);
-    for (int64_t i = a; i < b; ++i) {
-        const int64_t y = target[i];
-        if (y != ignore_index && y >= 0 && y < V) {
-            idx[off] = (int32_t)i;
-            pos[i] = off++;
-        } else {
-            pos[i] = -1;
+    for (int64_t i = a; i < b; i += 2) {
+        int64_t y[2];
+        pair_at(i, y[0], y[1]);
+        for (int k = 0; k < 2 && i + k < b; ++k) {
+            if (ok(y[k])) {
+                idx[off] = (int32_t)(i + k);
+                pos[i + k] = off++;
+            } else {
+                pos[i + k] = -1;
+            }
         }
     }
     if (threadIdx.x == T - 1) *count = off;
@@ -508,10 +555,17 @@ __global__ void k_zero_if_none(const int32_t* count, void* dst, int64_t bytes16)
 __global__ void k_count_valid_only(const int64_t* __restrict__ target, int64_t N, int64_t V,
                                    int64_t ignore_index, int32_t* count) {
     int valid = 0;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t y = target[i];
-        if (y != ignore_index && y >= 0 && y < V) ++valid;
+    auto take = [&](int64_t y) { valid += (y != ignore_index && y >= 0 && y < V) ? 1 : 0; };
+    const TargetPairs tp(target, N);
+    const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (int64_t i = tid; i < tp.n_pairs; i += (int64_t)gridDim.x * blockDim.x) {
+        const longlong2 v = tp.pairs[i];
+        take(v.x);
+        take(v.y);
+    }
+    if (tid == 0) {
+        if (tp.head != nullptr) take(*tp.head);
+        if (tp.tail != nullptr) take(*tp.tail);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) valid += __shfl_xor_sync(0xffffffffu, valid, o);
@@ -550,28 +604,96 @@ struct MergeParams {
     float* row_lse2;          // [chunk] for sweep 2 (null in forward-only mode)
     float* row_gcoef;
     int32_t* row_y;
+    // 1 when target, p_mask and every per-token output above start on a
+    // 16-byte boundary: groups of four rows then move as 128-bit vectors
+    int vec;
 };
 
-// Split-V merge: lse = M + log sum_k l_k 2^(m_k - M) (logsumexp_fwd's second
-// logsumexp; the tensor-parallel tutorial's sum of per-shard denominators),
-// then the per-token loss (cross_entropy_kernel step 4 and the
-// label-smoothing block) and the per-token gradient coefficient.
+// What the merge writes for one token.
+struct MergedRow {
+    float loss, lse, lse2, gcoef;
+    int32_t am, y;            // argmax; validated shard-local target or -1
+};
+
 // Threads per row of the split-V merge: each takes every kMergeSub-th vocab
 // tile in one online pass; the kMergeSub partial (max, sum) pairs of a row are
 // then combined with shuffles in a fixed order (deterministic).
 constexpr int kMergeSub = 8;
 
+// The per-token outputs of row m from its merged statistics (base-2 maximum
+// M2 and sum L, best vocabulary tile, sum of raw logits): the loss of
+// cross_entropy_kernel step 4 with the label-smoothing block, and the
+// gradient coefficient of steps 5-6.  y and pm are the row's target and
+// p_mask (pm is read only for a token that carries a loss).
+__device__ __forceinline__ MergedRow merge_finish_row(const MergeParams& p, int m, float M2,
+                                                      float L, int kbest, float szs, int64_t y,
+                                                      float pm) {
+    const int64_t gm = p.stats_row0 + m;
+    const bool valid = (y != p.ignore_index) && y >= 0 && y < p.Vtot;
+    const bool local_y = valid && y - p.v0 >= 0 && y - p.v0 < p.V;
+    float zyv = 0.f, szv = 0.f;
+    int32_t am = -1;
+    if (p.mode != MERGE_GATHERED) {
+        if (local_y) zyv = p.zy[m];
+        szv = p.s * szs;
+        if (p.part_am != nullptr) am = p.part_am[(size_t)kbest * p.ld_part + m] + (int32_t)p.v0;
+    } else {
+        // every shard's statistics, merged in shard order (split softmax:
+        // lse = M + log2 sum_r l_r 2^(m_r - M); the target logit and the
+        // logit sums add over shards; ties go to the lowest shard)
+        int rbest = 0;
+        for (int r = 0; r < p.n_shards; ++r) {
+            const float v = p.all_stats[((size_t)r * p.stats_N + gm) * 8];
+            if (v > M2) { M2 = v; rbest = r; }
+        }
+        for (int r = 0; r < p.n_shards; ++r) {
+            const float* st = p.all_stats + ((size_t)r * p.stats_N + gm) * 8;
+            L += st[1] * exp2f(st[0] - M2);
+            zyv += st[2];
+            szv += st[3];
+        }
+        am = __float_as_int(p.all_stats[((size_t)rbest * p.stats_N + gm) * 8 + 4]);
+    }
+    MergedRow o;
+    o.lse2 = M2 + log2f(L);
+    o.lse = o.lse2 * 0.69314718055994530942f;
+    o.am = am;
+    o.loss = 0.f;
+    o.gcoef = 0.f;
+    if (valid) {
+        const float T = p.total > 0.f ? p.total
+                        : (float)(p.count_dev != nullptr ? *p.count_dev : p.cnt->n_valid);
+        const float coef = 1.f / (pm * T);
+        // lse - z_y taken in base 2, where both carry the same rounding of
+        // acc * s * log2(e) (exactly 0 when the target is the only column)
+        float ce = (o.lse2 - zyv) * 0.69314718055994530942f;
+        if (p.eps > 0.f) ce = (1.f - p.eps) * ce + p.eps * (o.lse - szv / (float)p.Vtot);
+        o.loss = ce * coef;
+        o.gcoef = p.grad_out * p.s * coef;
+    }
+    o.y = local_y ? (int32_t)(y - p.v0) : -1;
+    return o;
+}
+
+// Split-V merge: lse = M + log sum_k l_k 2^(m_k - M) (logsumexp_fwd's second
+// logsumexp; the tensor-parallel tutorial's sum of per-shard denominators),
+// then the per-token loss (cross_entropy_kernel step 4 and the
+// label-smoothing block) and the per-token gradient coefficient.
+//
+// A warp covers four consecutive rows (8 lanes each).  Where the four rows
+// are all live and the pointers allow it, the warp reads their targets as two
+// longlong2 and their p_mask as one float4, and writes each per-token output
+// of the four rows as one 128-bit store, a different lane per output;
+// otherwise the first lane of each row reads and writes its row alone.
 __global__ void __launch_bounds__(256) k_merge_rows(MergeParams p) {
     const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+    const int lane = threadIdx.x & 31;
     const int m = tid / kMergeSub;
     const int g = tid % kMergeSub;
-    bool live = m < p.rows;
-    bool dead_dyn = false;
-    if (live && p.dyn_count != nullptr && m >= *p.dyn_count - p.dyn_base) {
-        live = false;
-        dead_dyn = true;
-    }
-    const int64_t gm = p.stats_row0 + m;          // token index within the call
+    const int live_rows = p.dyn_count != nullptr
+                              ? max(0, min(p.rows, *p.dyn_count - p.dyn_base)) : p.rows;
+    const bool live = m < live_rows;
+    const bool dead_dyn = m < p.rows && !live;
     float M2 = -CUDART_INF_F, L = 0.f, szs = 0.f;
     int kbest = 0x7fffffff;
     if (live && p.mode != MERGE_GATHERED) {
@@ -602,6 +724,47 @@ __global__ void __launch_bounds__(256) k_merge_rows(MergeParams p) {
         M2 = Mn;
         szs += so;
     }
+
+    // the same for every lane of the warp: its four rows are all live
+    const int m0 = m & ~3;
+    const bool vec = p.vec != 0 && p.mode != MERGE_EMIT_STATS && m0 + 3 < live_rows;
+    if (vec) {
+        const uint32_t full = 0xffffffffu;
+        const int r = lane >> 3;                 // this lane's row within the four
+        longlong2 tq = make_longlong2(0, 0);
+        float4 pq = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (lane == 1 || lane == 2) tq = reinterpret_cast<const longlong2*>(p.target + m0)[lane - 1];
+        if (lane == 0 && p.p_mask != nullptr) pq = *reinterpret_cast<const float4*>(p.p_mask + m0);
+        // rows 0, 1 come from lane 1's pair, rows 2, 3 from lane 2's
+        const long long t0 = __shfl_sync(full, tq.x, 1), t1 = __shfl_sync(full, tq.y, 1);
+        const long long t2 = __shfl_sync(full, tq.x, 2), t3 = __shfl_sync(full, tq.y, 2);
+        const float q0 = __shfl_sync(full, pq.x, 0), q1 = __shfl_sync(full, pq.y, 0);
+        const float q2 = __shfl_sync(full, pq.z, 0), q3 = __shfl_sync(full, pq.w, 0);
+        const int64_t y = r == 0 ? t0 : (r == 1 ? t1 : (r == 2 ? t2 : t3));
+        const float pm = r == 0 ? q0 : (r == 1 ? q1 : (r == 2 ? q2 : q3));
+        const MergedRow o = merge_finish_row(p, m, M2, L, kbest, szs, y, pm);
+        auto g4f = [&](float v) {
+            return make_float4(__shfl_sync(full, v, 0), __shfl_sync(full, v, 8),
+                               __shfl_sync(full, v, 16), __shfl_sync(full, v, 24));
+        };
+        auto g4i = [&](int32_t v) {
+            return make_int4(__shfl_sync(full, v, 0), __shfl_sync(full, v, 8),
+                             __shfl_sync(full, v, 16), __shfl_sync(full, v, 24));
+        };
+        const float4 loss4 = g4f(o.loss), lse4 = g4f(o.lse);
+        const float4 l24 = g4f(o.lse2), gc4 = g4f(o.gcoef);
+        const int4 am4 = g4i(o.am), y4 = g4i(o.y);
+        if (lane == 0) *reinterpret_cast<float4*>(p.loss_tok + m0) = loss4;
+        if (lane == 1 && p.lse_out != nullptr) *reinterpret_cast<float4*>(p.lse_out + m0) = lse4;
+        if (lane == 2 && p.am_out != nullptr) *reinterpret_cast<int4*>(p.am_out + m0) = am4;
+        if (p.row_lse2 != nullptr) {
+            if (lane == 3) *reinterpret_cast<float4*>(p.row_lse2 + m0) = l24;
+            if (lane == 4) *reinterpret_cast<float4*>(p.row_gcoef + m0) = gc4;
+            if (lane == 5) *reinterpret_cast<int4*>(p.row_y + m0) = y4;
+        }
+        return;
+    }
+
     if (g != 0 || m >= p.rows) return;
     if (dead_dyn) {
         // past the compacted tokens: no loss, zero gradient row
@@ -615,72 +778,50 @@ __global__ void __launch_bounds__(256) k_merge_rows(MergeParams p) {
     }
     const int64_t y = p.target[m];
     const bool valid = (y != p.ignore_index) && y >= 0 && y < p.Vtot;
-    const bool local_y = valid && y - p.v0 >= 0 && y - p.v0 < p.V;
-    float zyv = 0.f, szv = 0.f;
-    int32_t am = -1;
-    if (p.mode != MERGE_GATHERED) {
-        if (local_y) zyv = p.zy[m];
-        szv = p.s * szs;
-        if (p.part_am != nullptr) am = p.part_am[(size_t)kbest * p.ld_part + m] + (int32_t)p.v0;
-        if (p.mode == MERGE_EMIT_STATS) {
-            float* o = p.stats_out + (size_t)gm * 8;
-            o[0] = M2;
-            o[1] = L;
-            o[2] = zyv;
-            o[3] = szv;
-            o[4] = __int_as_float(am);
-            return;
-        }
-    } else {
-        // every shard's statistics, merged in shard order (split softmax:
-        // lse = M + log2 sum_r l_r 2^(m_r - M); the target logit and the
-        // logit sums add over shards; ties go to the lowest shard)
-        int rbest = 0;
-        for (int r = 0; r < p.n_shards; ++r) {
-            const float v = p.all_stats[((size_t)r * p.stats_N + gm) * 8];
-            if (v > M2) { M2 = v; rbest = r; }
-        }
-        for (int r = 0; r < p.n_shards; ++r) {
-            const float* st = p.all_stats + ((size_t)r * p.stats_N + gm) * 8;
-            L += st[1] * exp2f(st[0] - M2);
-            zyv += st[2];
-            szv += st[3];
-        }
-        am = __float_as_int(p.all_stats[((size_t)rbest * p.stats_N + gm) * 8 + 4]);
+    const float pm = (valid && p.p_mask != nullptr) ? p.p_mask[m] : 1.f;
+    if (p.mode == MERGE_EMIT_STATS) {
+        // this shard's statistics of the token: 32 bytes, two 128-bit stores
+        const bool local_y = valid && y - p.v0 >= 0 && y - p.v0 < p.V;
+        const int32_t am = p.part_am != nullptr
+                               ? p.part_am[(size_t)kbest * p.ld_part + m] + (int32_t)p.v0 : -1;
+        float4* o = reinterpret_cast<float4*>(p.stats_out + (size_t)(p.stats_row0 + m) * 8);
+        o[0] = make_float4(M2, L, local_y ? p.zy[m] : 0.f, p.s * szs);
+        o[1] = make_float4(__int_as_float(am), 0.f, 0.f, 0.f);
+        return;
     }
-    const float lse2 = M2 + log2f(L);
-    const float lse = lse2 * 0.69314718055994530942f;
-    float loss = 0.f, gcoef = 0.f;
-    if (valid) {
-        const float T = p.total > 0.f ? p.total
-                        : (float)(p.count_dev != nullptr ? *p.count_dev : p.cnt->n_valid);
-        const float pm = p.p_mask != nullptr ? p.p_mask[m] : 1.f;
-        const float coef = 1.f / (pm * T);
-        // lse - z_y taken in base 2, where both carry the same rounding of
-        // acc * s * log2(e) (exactly 0 when the target is the only column)
-        float ce = (lse2 - zyv) * 0.69314718055994530942f;
-        if (p.eps > 0.f) ce = (1.f - p.eps) * ce + p.eps * (lse - szv / (float)p.Vtot);
-        loss = ce * coef;
-        gcoef = p.grad_out * p.s * coef;
-    }
-    p.loss_tok[m] = loss;
-    if (p.lse_out != nullptr) p.lse_out[m] = lse;
-    if (p.am_out != nullptr) p.am_out[m] = am;
+    const MergedRow o = merge_finish_row(p, m, M2, L, kbest, szs, y, pm);
+    p.loss_tok[m] = o.loss;
+    if (p.lse_out != nullptr) p.lse_out[m] = o.lse;
+    if (p.am_out != nullptr) p.am_out[m] = o.am;
     if (p.row_lse2 != nullptr) {
-        p.row_lse2[m] = lse2;
-        p.row_gcoef[m] = gcoef;
-        p.row_y[m] = local_y ? (int32_t)(y - p.v0) : -1;
+        p.row_lse2[m] = o.lse2;
+        p.row_gcoef[m] = o.gcoef;
+        p.row_y[m] = o.y;
     }
 }
 
 // loss = sum_n loss[n] in a fixed order (one block, fp64 partials), so the
 // scalar is bit-reproducible run to run; also publishes the malformed-target
 // count and the device error bits (a timed-out wait) in err_count[0..1].
+// The per-token losses are read as float4 from the first 16-byte boundary
+// on; the up to three elements before it and the ragged end are added by
+// thread 0.
 __global__ void k_finish(const float* __restrict__ loss_tok, int64_t N, const Counters* cnt,
                          float* loss, int32_t* err_count) {
     __shared__ double red[1024];
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(loss_tok) & 15u;
+    const int64_t h = min(N, mis != 0 ? (int64_t)((16u - mis) / 4u) : (int64_t)0);
+    const int64_t n4 = (N - h) / 4;
+    const float4* q = reinterpret_cast<const float4*>(loss_tok + h);
     double acc = 0.0;
-    for (int64_t i = threadIdx.x; i < N; i += blockDim.x) acc += (double)loss_tok[i];
+    for (int64_t i = threadIdx.x; i < n4; i += blockDim.x) {
+        const float4 v = q[i];
+        acc += ((double)v.x + (double)v.y) + ((double)v.z + (double)v.w);
+    }
+    if (threadIdx.x == 0) {
+        for (int64_t i = 0; i < h; ++i) acc += (double)loss_tok[i];
+        for (int64_t i = h + 4 * n4; i < N; ++i) acc += (double)loss_tok[i];
+    }
     red[threadIdx.x] = acc;
     __syncthreads();
     for (int w = blockDim.x / 2; w > 0; w >>= 1) {

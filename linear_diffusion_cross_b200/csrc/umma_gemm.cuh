@@ -34,8 +34,9 @@
 // Operands are consumed K-major or MN-major straight from row-major HBM
 // through the tensor maps; no transposed copy of any operand is made.  Loads
 // carry no cluster multicast.  Every mbarrier wait is bounded by global time;
-// on time-out the CTA records FLDCE_DEV_ERR_TIMEOUT, stops issuing work and
-// frees its TMEM.
+// on time-out the CTA records FLDCE_DEV_ERR_TIMEOUT, stops issuing work,
+// waits (bounded again) for the MMAs and loads it already issued, and frees
+// its TMEM.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -205,7 +206,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* epi_smem = smem + S * Cfg::STAGE_BYTES;
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + Cfg::EPI_BYTES);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -218,6 +219,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
     auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * S + b); };
     auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * S + 2 + b); };
+    const uint32_t drain_bar = smem_u32(bars + 2 * S + 4);   // abort path only
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -228,6 +230,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(tfull_bar(b), 1);
             mbar_init(tempty_bar(b), 8);       // 4 epilogue warps x 2 CTAs
         }
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -271,13 +274,14 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         k1 = min(geom.k_iters, k0 + kps);
     };
 
+    uint32_t loads_issued = 0;                 // producer: stages loaded so far
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
         // evict_first on the streamed operand / evict_last on the reused one
         // measured more HBM traffic than the default priority, not less
         const uint64_t pol = l2_policy_evict_normal();
         const uint32_t lead_full0 = mapa_shared(full_bar(0), 0);
-        uint32_t it = 0;
+        uint32_t& it = loads_issued;
         bool ok = true;
         for (int u = pair; ok && u < units && !*abort_flag; u += npairs) {
             int mt, nt, split, k0, k1;
@@ -402,6 +406,28 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // A wait timed out somewhere in the pair.  Before TMEM is freed and
+        // the CTAs exit, let the asynchronous work already issued finish
+        // (each wait again bounded): the leader's MMA lane commits every MMA
+        // it issued to a local barrier and waits for it, and the leader's
+        // producer lane waits until the loads of the last S stages it issued
+        // (both CTAs' bytes are counted on its barriers) have landed.  The
+        // results of the call are invalid either way (FLDCE_DEV_ERR_TIMEOUT).
+        if (rank == 0 && warp == 1 && lane == 0) {
+            // (cta_group::2 like every tcgen05 op of this kernel; leader only)
+            tc_commit_pair_mc(drain_bar, 0x1);
+            mbar_wait_bounded(drain_bar, 0u, kWaitLimitNs);
+        }
+        if (rank == 0 && warp == 0 && lane == 0) {
+            const uint32_t first = loads_issued > (uint32_t)S ? loads_issued - S : 0u;
+            for (uint32_t i = first; i < loads_issued; ++i)
+                mbar_wait_bounded(full_bar((int)(i % S)), (i / S) & 1u, kWaitLimitNs);
+        }
+        __syncwarp();
+        tc_fence_before();
+        __syncthreads();
+    }
     cluster_sync();            // every MMA of the pair has completed and been read
     if (warp == 1) {
         tc_fence_after();

@@ -44,6 +44,7 @@ class Workload:
     total: float = 0.0         # > 0: explicit; <= 0: count of non-ignored tokens
     grad_out: float = 1.0
     chunk_n: int = 0           # 0: the library picks the token-chunk size
+    peaky_rows: Optional[torch.Tensor] = None   # W rows drawn x peaky_mult (sorted), or None
 
     @property
     def N(self) -> int:
@@ -131,9 +132,11 @@ def make(recipe: Recipe | str, seed: int = 0, *, batch: Optional[int] = None,
     g = torch.Generator().manual_seed(seed)
     H = torch.randn(N, D_, generator=g).to(dt)
     W = (recipe.sigma_w * torch.randn(V_, D_, generator=g)).to(dt)
+    peaky = None
     if recipe.peaky_frac > 0.0:
         rows = torch.randperm(V_, generator=g)[: max(1, int(V_ * recipe.peaky_frac))]
         W[rows] *= recipe.peaky_mult          # a power of two: exact in bf16
+        peaky = torch.sort(rows).values
     if recipe.t_block > 0:
         n_blocks = -(-N // recipe.t_block)
         t_unit = recipe.t_lo + (1.0 - recipe.t_lo) * torch.rand(n_blocks, generator=g)
@@ -151,7 +154,7 @@ def make(recipe: Recipe | str, seed: int = 0, *, batch: Optional[int] = None,
         p_mask=p_mask, logit_scale=recipe.logit_scale,
         label_smoothing=recipe.label_smoothing,
         total=0.0 if recipe.total_is_count else float(N),
-        chunk_n=recipe.chunk_n,
+        chunk_n=recipe.chunk_n, peaky_rows=peaky,
     )
     for k, v in overrides.items():
         if not hasattr(wl, k):

@@ -78,3 +78,55 @@ def test_comment_edits_keep_the_source_hash(tmp_path, monkeypatch):
     assert bench.source_hash() != h1
     f.write_text('int a = 1; const char* s = "// changed";\n')
     assert bench.source_hash() != h1
+
+
+def _env_without_launcher():
+    import os
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "LOCAL_WORLD_SIZE", "MASTER_ADDR",
+              "MASTER_PORT", "GROUP_RANK", "ROLE_RANK", "TORCHELASTIC_RUN_ID"):
+        env.pop(k, None)
+    env["OMP_NUM_THREADS"] = "1"
+    return env
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` with no external launcher starts two ranks through
+    torch.distributed.run; rank 0 prints the one JSON line with n_gpus 2 (the
+    reference arm, which needs no GPU: rank 0 times the oracle, rank 1 exits
+    without work)."""
+    import json
+    import subprocess
+    import sys
+    cmd = [sys.executable, bench.__file__, "--gpus", "2", "--impl", "reference",
+           "--workload", "tiny", "--steps", "1", "--warmup", "3", "--ref-tokens", "8"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=600,
+                         env=_env_without_launcher())
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(x) for x in res.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+    assert line["config"]["parallelism"] == "dp2"
+    assert line["steps"] == 1 and line["warmup"] == 3
+
+
+def test_gpus_flag_must_match_an_external_launcher(monkeypatch):
+    import pytest
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.world_from_env(2) == (2, 1, 1)
+    with pytest.raises(SystemExit):
+        bench.world_from_env(4)
+    monkeypatch.delenv("WORLD_SIZE")
+    assert bench.world_from_env(1)[0] == 1
+
+
+def test_both_arms_name_the_same_config():
+    from linear_diffusion_cross_b200 import synth
+    for name, r in synth.RECIPES.items():
+        c1 = bench.run_config(name, r, 1)
+        assert c1 == bench.run_config(name, r, 1)
+        assert set(c1) == {"workload", "N", "D", "V", "parallelism", "l2"}
+    assert "no flush" in bench.run_config("headline", synth.RECIPES["headline"], 1)["l2"]

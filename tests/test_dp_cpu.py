@@ -115,3 +115,57 @@ def test_accumulating_plan_is_refused():
     kernels = SimpleNamespace(plan=SimpleNamespace(dw_accumulate=True))
     with pytest.raises(ValueError):
         fwd_bwd_data_parallel(kernels, None, None, None, None, total=1.0)
+
+
+# ------------------------------------------------------------ a rank that leaves
+PG_TIMEOUT_S = 5
+
+
+def _leaver_worker(rank, port, outdir, total):
+    """Both ranks run one data-parallel step; then rank 1 leaves (exits
+    between steps, with no collective in flight) and rank 0 starts a second
+    step.  Rank 0 records whether that step raised, and how long it took."""
+    import datetime
+    import sys
+    import time
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from linear_diffusion_cross_b200.dp import fwd_bwd_data_parallel
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=WORLD, timeout=datetime.timedelta(seconds=PG_TIMEOUT_S))
+    H, W, y, p, _ = _case()
+    N = H.shape[0]
+    sl = slice(rank * N // WORLD, (rank + 1) * N // WORLD)
+    k = OracleKernels(W.shape[0], dict(logit_scale=1.0, label_smoothing=0.0, ignore_index=-100))
+    args = (k, torch.from_numpy(H[sl]), torch.from_numpy(W), torch.from_numpy(y[sl]),
+            torch.from_numpy(p[sl]))
+    fwd_bwd_data_parallel(*args, total=total)
+    dist.barrier()                       # step 1 is complete on both ranks
+    if rank == 1:
+        os._exit(0)                      # leaves without tearing down the group
+    time.sleep(0.5)                      # the peer is gone before step 2 starts
+    t0 = time.monotonic()
+    try:
+        fwd_bwd_data_parallel(*args, total=total)
+        outcome = "completed"
+    except Exception as e:              # gloo reports the lost peer or the timeout
+        outcome = type(e).__name__ + ": " + str(e).splitlines()[0][:200]
+    dt = time.monotonic() - t0
+    with open(os.path.join(outdir, "rank0.txt"), "w") as f:
+        f.write(f"{dt}\n{outcome}\n")
+    os._exit(0)                          # the group is broken: skip its teardown
+
+
+@pytest.mark.parametrize("total", [0.0, 11.0])
+def test_rank_leaving_between_steps_fails_the_next_step(total):
+    """The host-side form of failure detection in the data-parallel step: when
+    a rank leaves between steps, the surviving rank's next collective ends
+    with an error within the process group's timeout instead of hanging.
+    (total <= 0 fails on the count's all-reduce before any kernel; an explicit
+    total fails after the local step, on the dW reduction.)"""
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_leaver_worker, args=(_free_port(), d, total), nprocs=WORLD,
+                           join=True, start_method="spawn")
+        with open(os.path.join(d, "rank0.txt")) as f:
+            dt, outcome = f.read().splitlines()[:2]
+    assert outcome != "completed", "the step completed without its peer"
+    assert float(dt) < 6 * PG_TIMEOUT_S, f"took {dt} s to fail: {outcome}"

@@ -1,8 +1,16 @@
 """GPU parity at the full workload sizes, in the launch configuration bench.py
 times (default chunking, argmax on).  The oracle computes what it can one
-row at a time: every sampled token's lse, loss and dH row, every sampled
-vocabulary row of dW where the whole batch's lse is affordable (mid and
-headline), and properties that hold at any size everywhere:
+row at a time:
+
+* every sampled token's lse, loss and dH row;
+* for every workload, sampled vocabulary rows of dW, element by element:
+  always the last row (V - 1, the ragged tail of a vocabulary that is not a
+  multiple of the tile width), target rows of valid tokens, and for the
+  large workload a set of the rows drawn x8;
+* the scalar loss against the oracle's full-batch sum, and every token's
+  lse and per-token loss (the dW rows need the whole batch's lse anyway).
+
+Properties that hold at any size are checked everywhere as well:
 
 * ignored tokens: loss and dH row exactly zero (every token, not a sample);
 * loss == sum of loss_per_token;
@@ -17,8 +25,8 @@ import torch
 
 import oracle.fldce_oracle as O
 from linear_diffusion_cross_b200 import synth
-from tests._parity import (GRAD_TOL, LOSS_RTOL, check_rows, f64, maxabs_err, oracle_inputs,
-                           oracle_kw, run_gpu)
+from tests._parity import (GRAD_TOL, LOSS_RTOL, ROW_TOL, check_rows, f64, maxabs_err,
+                           oracle_inputs, oracle_kw, run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,19 +73,34 @@ def test_full_size(name):
     info.update(check_rows(wl, g, ref, rows, "bf16"))
     info["oracle_rows_s"] = time.time() - t1
 
-    if name in ("mid", "headline"):
-        must = [wl.V - 1] + [int(v) for v in y[valid][:8]]
-        vr = synth.sample_rows(wl.V, N_SAMPLE_VOCAB, 2, must).numpy()
-        t2 = time.time()
-        dWr, lse_all, lt_all = O.fldce_dw_rows(H, W, y, p, vr, total=T, **oracle_kw(wl))
-        info["oracle_dw_s"] = time.time() - t2
-        e_dw = maxabs_err(f64(g["dW"])[vr], dWr)
-        assert e_dw <= GRAD_TOL["bf16"], f"dW err {e_dw}"
-        info["dW"] = e_dw
-        loss_ref = float(lt_all.sum())
-        loss = float(g["loss"][0])
-        assert abs(loss - loss_ref) <= LOSS_RTOL * abs(loss_ref), (loss, loss_ref)
-        info["loss"] = abs(loss - loss_ref) / abs(loss_ref)
+    must = [wl.V - 1, wl.V - 2] + [int(v) for v in y[valid][:8]]
+    if wl.peaky_rows is not None:
+        # rows drawn x8: the peaky logits of the large workload
+        pk = wl.peaky_rows.numpy()
+        must += [int(v) for v in pk[np.linspace(0, pk.size - 1, 16).astype(np.int64)]]
+    vr = synth.sample_rows(wl.V, N_SAMPLE_VOCAB, 2, must).numpy()
+    t2 = time.time()
+    dWr, lse_all, lt_all = O.fldce_dw_rows(H, W, y, p, vr, total=T, **oracle_kw(wl))
+    info["oracle_dw_s"] = time.time() - t2
+    e_dw = maxabs_err(f64(g["dW"])[vr], dWr)
+    info["dW"] = e_dw
+    if wl.peaky_rows is not None:
+        pk_set = np.isin(vr, wl.peaky_rows.numpy())
+        info["dW_peaky_rows"] = int(pk_set.sum())
+        info["dW_peaky_err"] = maxabs_err(f64(g["dW"])[vr[pk_set]], dWr[pk_set])
+    assert e_dw <= GRAD_TOL["bf16"], f"dW err {e_dw}"
+    # every token: lse and per-token loss against the oracle's whole batch
+    e_lse = float(np.abs(g["lse"].double().numpy() - lse_all).max() /
+                  max(1.0, np.abs(lse_all).max()))
+    e_lt = maxabs_err(g["loss_per_token"].double().numpy(), lt_all)
+    info["lse_all"] = e_lse
+    info["loss_per_token_all"] = e_lt
+    assert e_lse <= ROW_TOL["bf16"], f"lse err {e_lse}"
+    assert e_lt <= ROW_TOL["bf16"], f"loss_per_token err {e_lt}"
+    loss_ref = float(lt_all.sum())
+    loss = float(g["loss"][0])
+    info["loss"] = abs(loss - loss_ref) / abs(loss_ref)
+    assert abs(loss - loss_ref) <= LOSS_RTOL * abs(loss_ref), (loss, loss_ref)
     print(name, info)
 
 

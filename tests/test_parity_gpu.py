@@ -8,8 +8,8 @@ import torch
 import oracle.fldce_oracle as O
 from linear_diffusion_cross_b200 import binding as B
 from linear_diffusion_cross_b200 import synth
-from tests._parity import (GRAD_TOL, LOSS_RTOL, check_rows, f64, maxabs_err, oracle_inputs,
-                           oracle_kw, run_gpu)
+from tests._parity import (ARGMAX_MARGIN, GRAD_TOL, LOSS_RTOL, ROW_TOL, check_rows, f64,
+                           maxabs_err, oracle_inputs, oracle_kw, run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -163,6 +163,19 @@ def test_forward_only_matches_fwd_bwd():
     assert torch.equal(f["lse"].cpu(), g["lse"])
     assert torch.equal(f["argmax"].cpu(), g["argmax"])
     assert torch.equal(f["loss_per_token"].cpu(), g["loss_per_token"])
+    # and directly against the float64 oracle
+    H, W, y, p = oracle_inputs(wl)
+    ref = O.fldce(H, W, y, p, total=wl.total, **oracle_kw(wl))
+    fl = float(f["loss"][0])
+    assert abs(fl - ref.loss) <= LOSS_RTOL * abs(ref.loss)
+    assert maxabs_err(f["loss_per_token"].double().cpu().numpy(), ref.loss_per_token) <= \
+        ROW_TOL["bf16"]
+    assert float(np.abs(f["lse"].double().cpu().numpy() - ref.lse).max()) <= \
+        ROW_TOL["bf16"] * max(1.0, float(np.abs(ref.lse).max()))
+    clear = ref.top2_gap > ARGMAX_MARGIN
+    assert np.array_equal(f["argmax"].cpu().numpy()[clear], ref.argmax[clear])
+    ign = y == wl.ignore_index
+    assert np.all(f["loss_per_token"].cpu().numpy()[ign] == 0.0)
 
 
 def test_error_codes_leave_outputs_untouched():

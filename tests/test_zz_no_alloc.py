@@ -11,6 +11,7 @@ process and after the rest of the suite.
 import pytest
 import torch
 
+import oracle.fldce_oracle as O
 from linear_diffusion_cross_b200 import binding as B
 from linear_diffusion_cross_b200 import synth
 from tests._parity import GRAD_TOL, LOSS_RTOL, ROW_TOL, maxabs_err
@@ -66,6 +67,17 @@ def test_noalloc_matches_workspace_entry_two_calls_in_a_row():
         results.append((got, ref))
     for got, ref in results:
         _compare(got, ref)
+    # and each call directly against the float64 oracle
+    for wl, (got, _) in zip(wls, results):
+        o = O.fldce(wl.H.double().numpy(), wl.W.double().numpy(), wl.target.numpy(),
+                    wl.p_mask.double().numpy(), total=wl.total, grad_out=1.5,
+                    label_smoothing=wl.label_smoothing)
+        assert abs(float(got["loss"][0]) - o.loss) <= LOSS_RTOL * abs(o.loss)
+        for k, want in (("dH", o.dH), ("dW", o.dW)):
+            e = maxabs_err(got[k].double().cpu().numpy(), want)
+            assert e <= GRAD_TOL["bf16"], (k, e)
+        e = maxabs_err(got["loss_per_token"].double().cpu().numpy(), o.loss_per_token)
+        assert e <= ROW_TOL["bf16"], e
 
 
 def test_noalloc_rejects_problems_beyond_the_static_scratch():
