@@ -300,6 +300,9 @@ def main():
                     help="also time torch.matmul (cuBLAS) on the step's three GEMM shapes")
     ap.add_argument("--no-skip", action="store_true",
                     help="do not time the FLDCE_FLAG_SKIP_IGNORED variant")
+    ap.add_argument("--fused-dh", action="store_true",
+                    help="the alternative design: sweep 2 fused with the dH GEMM "
+                         "(FLDCE_FLAG_FUSED_DH), G fed to dH from shared memory")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.gpus < 1:
@@ -320,7 +323,8 @@ def main():
     wl = synth.make(r, 0)
     N, D, V = wl.N, wl.D, wl.V
     plan = B.Plan(D, V, N, dtype=wl.H.dtype, chunk_N=wl.chunk_n, logit_scale=wl.logit_scale,
-                  label_smoothing=wl.label_smoothing, ignore_index=wl.ignore_index, device=dev)
+                  label_smoothing=wl.label_smoothing, ignore_index=wl.ignore_index,
+                  fused_dh=args.fused_dh, device=dev)
     H, W = wl.H.to(dev), wl.W.to(dev)
     y, p = wl.target.to(dev), wl.p_mask.to(dev)
     total = wl.total if wl.total > 0 else 0.0
@@ -402,7 +406,10 @@ def main():
     roof = None
     if dom in GEMM_KINDS:
         chunks = -(-N // B.fldce_chunk_size(plan.handle))
-        fl_launch = 2.0 * N * D * V / chunks
+        # GEMMs one launch of the kind performs (the fused kernel does the
+        # logit recompute and dH)
+        gemms = 2 if (args.fused_dh and dom == "g_sweep") else 1
+        fl_launch = gemms * 2.0 * N * D * V / chunks
         ach = fl_launch / (dom_ms / 1e3) / 1e12
         if wl.H.dtype == torch.bfloat16:
             roof = {"bound": "tensor", "kernel": dom, "achieved": ach,
@@ -480,6 +487,8 @@ def main():
             "dtype": "bf16" if wl.H.dtype == torch.bfloat16 else "f32",
             "data": "synthetic (seeded; shapes and masking of the workload)",
             "config": config, "chunk_N": B.fldce_chunk_size(plan.handle),
+            "design": ("fused sweep 2 + dH (G from shared memory)" if args.fused_dh else
+                       "staged G (sweep 2 writes G; separate dH and dW GEMMs)"),
             "tflops": world * flops / (ms / 1e3) / 1e12,
             "tflops_executed_8NDV": world * flops * 4 / 3 / (ms / 1e3) / 1e12,
             "pct_of_bf16_peak": 100.0 * flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],

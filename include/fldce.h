@@ -80,6 +80,17 @@ extern "C" {
  * and db as they are.  dH is still overwritten.  The pages always overwrite
  * (their dW is a fresh buffer per call); this flag is an extension. */
 #define FLDCE_FLAG_DW_ACCUMULATE 0x8u
+/* Sweep 2 fused with the dH GEMM (bf16 only, not with
+ * FLDCE_FLAG_SKIP_IGNORED): each 256 x 256 tile of the logit gradient G is
+ * formed in shared memory and fed from there, as the A operand, to the dH
+ * tensor-core MMAs, whose per-tile fp32 partials are reduce-added into an
+ * fp32 dH accumulator in the workspace; G still goes to HBM once, for the
+ * dW GEMM.  Same results as without the flag (up to the summation order of
+ * dH).  The page runs dx = dlogits @ weight on the gradient it wrote over
+ * the logits (fused_linear_cross_entropy_forward's chunk loop); this is the
+ * on-chip form of that step.  An alternative design, measured against the
+ * default (staged G read back by a separate dH GEMM), not the default. */
+#define FLDCE_FLAG_FUSED_DH      0x10u
 
 typedef struct fldce_plan* fldce_handle;
 

@@ -33,6 +33,7 @@ FLDCE_FLAG_DW_FP32 = 0x1
 FLDCE_FLAG_SKIP_IGNORED = 0x2
 FLDCE_FLAG_DH_FP32 = 0x4
 FLDCE_FLAG_DW_ACCUMULATE = 0x8
+FLDCE_FLAG_FUSED_DH = 0x10
 
 # every symbol include/fldce.h declares
 EXPORTS = ("fldce_create", "fldce_workspace_size", "fldce_chunk_size", "fldce_fwd_bwd",
@@ -319,7 +320,7 @@ class Plan:
                  chunk_N: int = 0, logit_scale: float = 1.0, label_smoothing: float = 0.0,
                  ignore_index: int = -100, dw_fp32: bool = False, skip_ignored: bool = False,
                  dh_fp32: bool = False, vocab_start: int = 0, vocab_total: int = 0,
-                 dw_accumulate: bool = False, device=None):
+                 dw_accumulate: bool = False, fused_dh: bool = False, device=None):
         code = FLDCE_BF16 if dtype == torch.bfloat16 else FLDCE_FP32
         if _TORCH_DTYPE[code] != dtype:
             raise TypeError(f"unsupported dtype {dtype}")
@@ -334,8 +335,10 @@ class Plan:
             flags=(FLDCE_FLAG_DW_FP32 if dw_fp32 else 0) |
             (FLDCE_FLAG_SKIP_IGNORED if skip_ignored else 0) |
             (FLDCE_FLAG_DH_FP32 if dh_fp32 else 0) |
-            (FLDCE_FLAG_DW_ACCUMULATE if dw_accumulate else 0),
+            (FLDCE_FLAG_DW_ACCUMULATE if dw_accumulate else 0) |
+            (FLDCE_FLAG_FUSED_DH if fused_dh else 0),
             vocab_start=vocab_start, vocab_total=vocab_total)
+        self.fused_dh = bool(fused_dh)
         self.dh_fp32 = bool(dh_fp32)
         self.dw_accumulate = bool(dw_accumulate)
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)

@@ -33,6 +33,7 @@
 #include <vector>
 
 #include "../../include/fldce.h"
+#include "fused_gdh.cuh"
 #include "kernels.cuh"
 
 using namespace fldce;
@@ -243,6 +244,41 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, int M, int64
     }
     const int pairs = std::min(g.num_tiles * g.k_splits, std::max(1, sms / 2));
     kern<<<2 * pairs, kGemmThreads, Cfg::SMEM_BYTES, st>>>(a, b, g, ep, err);
+    return cudaGetLastError();
+}
+
+// Sweep 2 fused with the dH GEMM (FLDCE_FLAG_FUSED_DH): G tiles to HBM
+// through gp.gmap, dH partials reduce-added into the fp32 map mDh.
+cudaError_t launch_fused_gdh(const CUtensorMap& mH, const CUtensorMap& mW, const CUtensorMap& mWmn,
+                             const CUtensorMap& mDh, int rows, int64_t V, int64_t D,
+                             const Walk& w, const GEpi::Params& gp, int32_t* err, int sms,
+                             cudaStream_t st) {
+    using Cfg = FusedGdhCfg;
+    GemmGeom g{};
+    g.tiles_m = (int)cdiv(rows, Cfg::PAIR_M);
+    g.tiles_n = (int)cdiv(V, Cfg::BN);
+    g.k_iters = (int)cdiv(D, Cfg::BK);
+    g.k_splits = 1;
+    g.num_tiles = g.tiles_m * g.tiles_n;
+    g.n_fastest = w.n_fastest;
+    g.group = w.group;
+    if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
+    auto kern = fused_gdh_kernel<Cfg>;
+    static std::atomic<uint64_t> attr_set{0};
+    int devid = 0;
+    cudaError_t e = cudaGetDevice(&devid);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = devid < 64 ? (uint64_t(1) << devid) : 0;
+    if (bit == 0 || (attr_set.load(std::memory_order_acquire) & bit) == 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Cfg::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit, std::memory_order_release);
+    }
+    const int pairs = std::min(g.num_tiles, std::max(1, sms / 2));
+    const int d_chunks = (int)cdiv(D, Cfg::DH_N);
+    kern<<<2 * pairs, kGemmThreads, Cfg::SMEM_BYTES, st>>>(mH, mW, mWmn, mDh, g, d_chunks, D, gp,
+                                                          err);
     return cudaGetLastError();
 }
 
@@ -663,9 +699,21 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             gp.eps_over_V = eps / (float)h->Vtot;
             gp.one_minus_eps = 1.f - eps;
             gp.bias = static_cast<const __nv_bfloat16*>(bias);
-            FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, sweep_walk, gp,
-                                                 &cnt->dev_err, dev.sms, st,
-                                                 DynRows{dynp, (int)r0, 1})));
+            const bool fused_dh = (cfg.flags & FLDCE_FLAG_FUSED_DH) != 0;
+            float* dh_part = reinterpret_cast<float*>(ws + L.dh_acc);
+            if (fused_dh) {
+                // sweep 2 and dH in one kernel: G from shared memory into the
+                // dH MMAs, fp32 partials reduce-added into dh_part
+                CUtensorMap mDh;
+                if (!make_store_map(&mDh, dh_part, D, rows, D, 4)) return FLDCE_ERR_CUDA;
+                FLDCE_CUDA(cudaMemsetAsync(dh_part, 0, (size_t)rows * D * 4, st));
+                FLDCE_CUDA(launch_fused_gdh(mH_k, mW_k, mW_mn, mDh, rows, V, D, sweep_walk, gp,
+                                            &cnt->dev_err, dev.sms, st));
+            } else {
+                FLDCE_CUDA((launch_gemm<CfgKK, GEpi>(mH_k, mW_k, rows, V, D, sweep_walk, gp,
+                                                     &cnt->dev_err, dev.sms, st,
+                                                     DynRows{dynp, (int)r0, 1})));
+            }
             prof_mark(h, PK_G, st);
             if (bias != nullptr) {
                 FLDCE_CUDA(launch_colsum(G, true, h->Vpad, rows, V, db_part, db_acc, ci > 0, st,
@@ -683,6 +731,15 @@ int run(fldce_handle h, const fldce_call& call, bool backward, int mode = MERGE_
             // split j stores its fp32 partial in its own buffer and one pass
             // sums them in split order (deterministic) into dH.
             auto do_dh = [&]() -> int {
+                if (fused_dh) {
+                    // the fused kernel left dH in fp32: round (or copy) it out
+                    const bool dh_fp32 = (cfg.flags & FLDCE_FLAG_DH_FP32) != 0;
+                    void* dHc = static_cast<uint8_t*>(dH) + (size_t)r0 * D * (dh_fp32 ? 4 : 2);
+                    FLDCE_CUDA(launch_sum_splits(dh_part, 0, 1, dHc, !dh_fp32, (int64_t)rows * D,
+                                                 dev.sms, st));
+                    prof_mark(h, PK_CONVERT, st);
+                    return FLDCE_OK;
+                }
                 const DhPlan dp = plan_dh(rows, D, V, std::max(1, dev.sms / 2));
                 const bool wide = dp.wide;
                 const int ks = dp.k_splits;
@@ -814,7 +871,10 @@ int fldce_create(fldce_handle* out, const fldce_config* cfg, size_t* workspace_b
     if (!std::isfinite(cfg->logit_scale) || cfg->logit_scale == 0.f) return FLDCE_ERR_INVALID_ARG;
     if (cfg->dtype != FLDCE_BF16 && cfg->dtype != FLDCE_FP32) return FLDCE_ERR_UNSUPPORTED;
     if ((cfg->flags & ~(FLDCE_FLAG_DW_FP32 | FLDCE_FLAG_SKIP_IGNORED | FLDCE_FLAG_DH_FP32 |
-                        FLDCE_FLAG_DW_ACCUMULATE)) != 0)
+                        FLDCE_FLAG_DW_ACCUMULATE | FLDCE_FLAG_FUSED_DH)) != 0)
+        return FLDCE_ERR_UNSUPPORTED;
+    if ((cfg->flags & FLDCE_FLAG_FUSED_DH) != 0 &&
+        (cfg->dtype != FLDCE_BF16 || (cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0))
         return FLDCE_ERR_UNSUPPORTED;
     if ((cfg->flags & FLDCE_FLAG_SKIP_IGNORED) != 0 &&
         (cfg->dtype != FLDCE_BF16 || (cfg->flags & FLDCE_FLAG_DH_FP32) != 0))

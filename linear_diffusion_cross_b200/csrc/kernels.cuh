@@ -256,63 +256,86 @@ struct GEpi {
         const __nv_bfloat16* bias;   // [V] or null
     };
 
-    template <class Cfg>
-    static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
-                                               const AccRow& acc, Stager& st) {
-        const int m = t.row0 + t.row;
-        const int64_t n0 = t.col0;
-        float gc = 0.f, L2 = 0.f;
-        int yrel = -1;
-        if (m < (t.rows_dyn >= 0 ? t.rows_dyn : p.rows)) {
-            gc = p.gcoef[m];
-            if (gc != 0.f) {
-                L2 = p.lse2[m];
+    // What one thread needs for its row of a vocabulary tile starting at n0.
+    struct Row {
+        float gc, L2, base, tcorr;
+        int yrel, ncols;
+    };
+
+    template <int BN>
+    static __device__ __forceinline__ Row row_setup(const Params& p, int m, int rows_dyn,
+                                                    int64_t n0) {
+        Row w;
+        w.gc = 0.f;
+        w.L2 = 0.f;
+        w.yrel = -1;
+        if (m < (rows_dyn >= 0 ? rows_dyn : p.rows)) {
+            w.gc = p.gcoef[m];
+            if (w.gc != 0.f) {
+                w.L2 = p.lse2[m];
                 const int y = p.ycol[m];
-                if (y >= n0 && y < n0 + Cfg::BN) yrel = (int)(y - n0);
+                if (y >= n0 && y < n0 + BN) w.yrel = (int)(y - n0);
             }
         }
-        const float base = gc * p.eps_over_V;
-        const float tcorr = gc * p.one_minus_eps;
-        const int ncols = (int)((p.V - n0) < Cfg::BN ? (p.V - n0) : Cfg::BN);
-        static_assert(Cfg::NSUB == 1, "one 256-column MMA per vocabulary tile");
-        for_each_chunk<Cfg::NCHUNK>(acc, [&](const uint32_t (&r)[32], int j) {
-            float g[32];
-            if (p.bias != nullptr) {
-                float b[32];
-                load_bias32(p.bias, n0 + 32 * j, p.V, b);
+        w.base = w.gc * p.eps_over_V;
+        w.tcorr = w.gc * p.one_minus_eps;
+        w.ncols = (int)((p.V - n0) < BN ? (p.V - n0) : BN);
+        return w;
+    }
+
+    // G of columns [n0 + 32 j, n0 + 32 j + 32) of the row from its raw
+    // accumulator values r (bias added first when there is one).
+    static __device__ __forceinline__ void chunk(const Params& p, const Row& w,
+                                                 const uint32_t (&r)[32], int64_t n0, int j,
+                                                 float (&g)[32]) {
+        const float gc = w.gc, L2 = w.L2, base = w.base;
+        if (p.bias != nullptr) {
+            float b[32];
+            load_bias32(p.bias, n0 + 32 * j, p.V, b);
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float a0, a1, t0, t1;
-                    add2(a0, a1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), b[i], b[i + 1]);
-                    fma2(t0, t1, a0, a1, p.c, p.c, -L2, -L2);
-                    fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
-                }
-                if (gc == 0.f) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) g[i] = 0.f;
-                }
-            } else if (gc != 0.f) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float t0, t1;
-                    fma2(t0, t1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.c, p.c, -L2,
-                         -L2);
-                    fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
-                }
-            } else {
+            for (int i = 0; i < 32; i += 2) {
+                float a0, a1, t0, t1;
+                add2(a0, a1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), b[i], b[i + 1]);
+                fma2(t0, t1, a0, a1, p.c, p.c, -L2, -L2);
+                fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
+            }
+            if (gc == 0.f) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) g[i] = 0.f;
             }
-            if ((unsigned)(yrel - 32 * j) < 32u) {
+        } else if (gc != 0.f) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (i == yrel - 32 * j) g[i] -= tcorr;
+            for (int i = 0; i < 32; i += 2) {
+                float t0, t1;
+                fma2(t0, t1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.c, p.c, -L2,
+                     -L2);
+                fma2(g[i], g[i + 1], gc, gc, ex2(t0), ex2(t1), -base, -base);
             }
-            if (32 * j + 32 > ncols) {
+        } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (32 * j + i >= ncols) g[i] = 0.f;
-            }
+            for (int i = 0; i < 32; ++i) g[i] = 0.f;
+        }
+        if ((unsigned)(w.yrel - 32 * j) < 32u) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (i == w.yrel - 32 * j) g[i] -= w.tcorr;
+        }
+        if (32 * j + 32 > w.ncols) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (32 * j + i >= w.ncols) g[i] = 0.f;
+        }
+    }
+
+    template <class Cfg>
+    static __device__ __forceinline__ void run(const Params& p, const TileCtx& t,
+                                               const AccRow& acc, Stager& st) {
+        const int64_t n0 = t.col0;
+        const Row w = row_setup<Cfg::BN>(p, t.row0 + t.row, t.rows_dyn, n0);
+        static_assert(Cfg::NSUB == 1, "one 256-column MMA per vocabulary tile");
+        for_each_chunk<Cfg::NCHUNK>(acc, [&](const uint32_t (&r)[32], int j) {
+            float g[32];
+            chunk(p, w, r, n0, j, g);
             if ((j & 1) == 0) st.acquire();
             stage_bf16_half(st, j, g);
             if (j & 1) st.flush(&p.gmap, (int)(n0 + 32 * (j - 1)), t.row0 + 32 * t.q, false);

@@ -124,6 +124,34 @@ __device__ __forceinline__ int apply_dyn_rows(GemmGeom& g) {
     return n;
 }
 
+// Coordinates of unit u of the persistent walk: output tile (mt, nt), K
+// split and its K-step range [k0, k1) (kps = K steps per split).  Units of
+// one split cover the tiles in blocks of `group` tiles along the fast
+// dimension: every tile of a block along the slow dimension, then the next
+// block.
+__device__ __forceinline__ void walk_unit(const GemmGeom& g, int kps, int u, int& mt, int& nt,
+                                          int& split, int& k0, int& k1) {
+    const int n_fast = g.n_fastest ? g.tiles_n : g.tiles_m;
+    const int n_slow = g.n_fastest ? g.tiles_m : g.tiles_n;
+    const int grp = max(1, min(g.group, n_fast));
+    split = u / g.num_tiles;
+    const int tile = u - split * g.num_tiles;
+    const int blk = tile / (grp * n_slow);
+    const int r = tile - blk * (grp * n_slow);
+    const int f0 = blk * grp;
+    const int gb = min(grp, n_fast - f0);          // the last block may be narrower
+    const int f = f0 + r % gb, sl = r / gb;
+    if (g.n_fastest) {
+        nt = f;
+        mt = sl;
+    } else {
+        mt = f;
+        nt = sl;
+    }
+    k0 = split * kps;
+    k1 = min(g.k_iters, k0 + kps);
+}
+
 // Where the current tile of this thread sits.
 struct TileCtx {
     int rows_dyn;         // live rows from the device-side count, or -1
@@ -252,26 +280,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         *abort_flag = 1;
         if (lane == 0) atomicOr(err, FLDCE_DEV_ERR_TIMEOUT);
     };
-    const int n_fast = geom.n_fastest ? geom.tiles_n : geom.tiles_m;
-    const int n_slow = geom.n_fastest ? geom.tiles_m : geom.tiles_n;
-    const int grp = max(1, min(geom.group, n_fast));
     auto unit_coords = [&](int u, int& mt, int& nt, int& split, int& k0, int& k1) {
-        split = u / geom.num_tiles;
-        const int tile = u - split * geom.num_tiles;
-        const int blk = tile / (grp * n_slow);
-        const int r = tile - blk * (grp * n_slow);
-        const int f0 = blk * grp;
-        const int gb = min(grp, n_fast - f0);          // the last block may be narrower
-        const int f = f0 + r % gb, sl = r / gb;
-        if (geom.n_fastest) {
-            nt = f;
-            mt = sl;
-        } else {
-            mt = f;
-            nt = sl;
-        }
-        k0 = split * kps;
-        k1 = min(geom.k_iters, k0 + kps);
+        walk_unit(geom, kps, u, mt, nt, split, k0, k1);
     };
 
     uint32_t loads_issued = 0;                 // producer: stages loaded so far

@@ -57,7 +57,7 @@ def test_version(lib):
     (dict(logit_scale=float("inf")), B.FLDCE_ERR_INVALID_ARG),
     (dict(D=60), B.FLDCE_ERR_UNSUPPORTED),
     (dict(dtype=7), B.FLDCE_ERR_UNSUPPORTED),
-    (dict(flags=0x10), B.FLDCE_ERR_UNSUPPORTED),
+    (dict(flags=0x20), B.FLDCE_ERR_UNSUPPORTED),
     (dict(dtype=1, flags=0x2), B.FLDCE_ERR_UNSUPPORTED),
 ])
 def test_create_rejects(lib, kw, code):
@@ -137,3 +137,21 @@ def test_strerror(lib):
     for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert B.fldce_strerror(code) and B.fldce_strerror(code) != "unknown status"
     assert B.fldce_strerror(-99) == "unknown status"
+
+
+def test_fused_dh_flag_combinations(lib):
+    # the fused sweep-2 + dH kernel is a bf16 tensor-core design and runs on
+    # every token (no compaction); its workspace is that of the staged design
+    h, ws_f = B.fldce_create(B.FLDCE_BF16, 2560, 151936, 8192, flags=B.FLDCE_FLAG_FUSED_DH)
+    B.fldce_destroy(h)
+    h, ws = B.fldce_create(B.FLDCE_BF16, 2560, 151936, 8192)
+    B.fldce_destroy(h)
+    assert ws_f == ws
+    for dtype, flags in ((B.FLDCE_FP32, B.FLDCE_FLAG_FUSED_DH),
+                         (B.FLDCE_BF16, B.FLDCE_FLAG_FUSED_DH | B.FLDCE_FLAG_SKIP_IGNORED)):
+        with pytest.raises(B.FldceError) as e:
+            B.fldce_create(dtype, 64, 512, 64, flags=flags)
+        assert e.value.status == B.FLDCE_ERR_UNSUPPORTED
+    h, _ = B.fldce_create(B.FLDCE_BF16, 64, 512, 64,
+                          flags=B.FLDCE_FLAG_FUSED_DH | B.FLDCE_FLAG_DH_FP32)
+    B.fldce_destroy(h)
