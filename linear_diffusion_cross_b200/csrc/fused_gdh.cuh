@@ -331,8 +331,9 @@ fused_gdh_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant_
 #pragma unroll
                     for (int b = 0; b < 4; ++b)
                         if (n0 + 64 * b < gp.V)
-                            tma_store_2d(&gp.gmap, gbase + b * Cfg::G_BLOCK_BYTES + q * 4096u,
-                                         (int)(n0 + 64 * b), row0 + 32 * q);
+                            tma_store_2d_hint(&gp.gmap, gbase + b * Cfg::G_BLOCK_BYTES + q * 4096u,
+                                              (int)(n0 + 64 * b), row0 + 32 * q,
+                                              l2_policy_evict_first());
                     bulk_commit_group();
                 }
             }
