@@ -47,10 +47,9 @@ class HostPipeline:
             })
         self.copy_stream = torch.cuda.Stream(device=dev)      # host -> device
         self.fetch_stream = torch.cuda.Stream(device=dev)     # device -> host
-        self.filled = [torch.cuda.Event() for _ in range(2)]
-        self.freed = [torch.cuda.Event() for _ in range(2)]
-        self.done = [torch.cuda.Event() for _ in range(2)]
-        self.fetched = [torch.cuda.Event() for _ in range(2)]
+        self.filled = [torch.cuda.Event() for _ in range(2)]    # inputs landed
+        self.done = [torch.cuda.Event() for _ in range(2)]      # the call finished
+        self.fetched = [torch.cuda.Event() for _ in range(2)]   # results downloaded
         self._last = 0
 
     @property
@@ -75,7 +74,7 @@ class HostPipeline:
     def _fill(self, slot: int, host: dict):
         s = self.slots[slot]
         cs = self.copy_stream
-        cs.wait_event(self.freed[slot])            # the call that read this slot is done
+        cs.wait_event(self.done[slot])             # the call that read this slot is done
         with torch.cuda.stream(cs):
             s["H"].copy_(host["H"], non_blocking=True)
             s["W"].copy_(host["W"], non_blocking=True)
@@ -90,7 +89,6 @@ class HostPipeline:
         stream.wait_event(self.fetched[slot])      # results of two steps ago are out
         self.plan.fwd_bwd(s["H"], s["W"], s["y"], s["p"], total, grad_out, out=s["out"],
                           stream=stream)
-        self.freed[slot].record(stream)
         self.done[slot].record(stream)
 
     def _fetch(self, slot: int, copies) -> None:
