@@ -261,7 +261,9 @@ cudaError_t launch_fused_gdh(const CUtensorMap& mH, const CUtensorMap& mW, const
     g.k_splits = 1;
     g.num_tiles = g.tiles_m * g.tiles_n;
     g.n_fastest = w.n_fastest;
-    g.group = w.group;
+    // token tiles in blocks whose fp32 dH rows (the reduce-add targets) and H
+    // panels stay in L2 together; W is read once per block
+    g.group = walk_group(g.tiles_m, (size_t)Cfg::PAIR_M * D * (4 + 2), kL2BudgetSweep);
     if (g.num_tiles == 0 || g.k_iters == 0) return cudaSuccess;
     auto kern = fused_gdh_kernel<Cfg>;
     static std::atomic<uint64_t> attr_set{0};

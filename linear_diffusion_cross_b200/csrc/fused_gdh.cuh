@@ -19,7 +19,9 @@
 //      M = 256, N = 128, K = 256 vocabulary rows, A = G from shared memory,
 //      B = W read MN-major.  Two 128-column TMEM accumulators alternate, so
 //      the epilogue flushes chunk j (fp32 TMA reduce-add into a dH
-//      accumulator) while the MMAs of chunk j + 1 run.
+//      accumulator) while the MMAs of chunk j + 1 run.  Each epilogue warp
+//      stages a whole chunk (four 32 x 32 fp32 boxes) before one proxy fence
+//      and one bulk group of four reduce-adds.
 // No dH accumulator fits on chip across the whole vocabulary (a 256 x D fp32
 // row block is 2.6 MB at D = 2560, TMEM holds 512 KB per pair), so each
 // unit's dH partial is flushed: 256 x D x 4 bytes of reduce-add traffic per
@@ -39,7 +41,7 @@
 namespace fldce {
 
 struct FusedGdhCfg {
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = 3;
     static constexpr int BM = 128;                 // token rows per CTA
     static constexpr int PAIR_M = 256;
     static constexpr int BN = 256;                 // vocabulary columns of a unit
@@ -51,8 +53,9 @@ struct FusedGdhCfg {
     static constexpr uint32_t DH_STAGE_BYTES = 64 * BK * 2;     // W [64 vocab][64 d], 8 KB
     static constexpr uint32_t G_BLOCK_BYTES = BM * 64 * 2;      // 64 vocabulary columns
     static constexpr uint32_t G_BYTES = 4 * G_BLOCK_BYTES;      // 64 KB
-    static constexpr uint32_t EPI_BUF_BYTES = 32 * 128;
-    static constexpr uint32_t EPI_BYTES = 4 * 2 * EPI_BUF_BYTES;
+    static constexpr uint32_t EPI_BUF_BYTES = 32 * 128;         // one 32 x 32 fp32 box
+    static constexpr uint32_t EPI_WARP_BYTES = (DH_N / 32) * EPI_BUF_BYTES;   // a whole chunk
+    static constexpr uint32_t EPI_BYTES = 4 * EPI_WARP_BYTES;
     static constexpr uint32_t BAR_BYTES = 256;
     static constexpr uint32_t SMEM_BYTES =
         1024 + STAGES * STAGE_BYTES + G_BYTES + EPI_BYTES + BAR_BYTES;
@@ -281,7 +284,15 @@ fused_gdh_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant_
         // ------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        Stager st{smem_u32(epi_smem) + (uint32_t)(q * 2) * Cfg::EPI_BUF_BYTES, lane, 0};
+        // this warp's four staging boxes, 128B-swizzled like the store maps
+        const uint32_t stage0 = smem_u32(epi_smem) + (uint32_t)q * Cfg::EPI_WARP_BYTES;
+        auto put_box = [&](int sub, const uint32_t (&r)[32]) {
+            const uint32_t line = stage0 + (uint32_t)sub * Cfg::EPI_BUF_BYTES + (uint32_t)lane * 128u;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                st_shared_v4(line + (uint32_t)((cc ^ (lane & 7)) << 4),
+                             make_uint4(r[4 * cc], r[4 * cc + 1], r[4 * cc + 2], r[4 * cc + 3]));
+        };
         const uint32_t lead_gready = mapa_shared(g_ready, 0);
         const uint32_t lead_dhe0 = mapa_shared(dh_empty(0), 0);
         const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
@@ -349,23 +360,17 @@ fused_gdh_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant_
                 }
                 tc_fence_after();
                 const uint32_t tcol = trow + Cfg::TM_DH + (uint32_t)(Cfg::DH_N * b);
+                // the previous chunk's reduce-adds (and the G stores) have read
+                // their shared-memory sources
+                if (lane == 0) bulk_wait_group_read<0>();
+                __syncwarp();
                 uint32_t ra[32], rb[32];
                 tmem_ld_32x32b_x32(tcol, ra);
                 tmem_ld_wait_regs(ra);
-                auto flush = [&](const uint32_t (&r)[32], int sub) {
-                    const int x = j * Cfg::DH_N + 32 * sub;
-                    if (!rows_live || x >= D) return;
-                    st.acquire();
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc)
-                        st.put(cc, make_uint4(r[4 * cc], r[4 * cc + 1], r[4 * cc + 2],
-                                              r[4 * cc + 3]));
-                    st.flush(&tmDh, x, row0 + 32 * q, true);
-                };
 #pragma unroll 1
                 for (int sub = 0; sub < Cfg::DH_N / 32; sub += 2) {
                     tmem_ld_32x32b_x32(tcol + 32u * (sub + 1), rb);
-                    flush(ra, sub);
+                    put_box(sub, ra);
                     tmem_ld_wait_regs(rb);
                     const bool more = sub + 2 < Cfg::DH_N / 32;
                     if (more) tmem_ld_32x32b_x32(tcol + 32u * (sub + 2), ra);
@@ -375,12 +380,26 @@ fused_gdh_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant_
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(lead_dhe0 + 8u * (uint32_t)b);
                     }
-                    flush(rb, sub + 1);
+                    put_box(sub + 1, rb);
                     if (more) tmem_ld_wait_regs(ra);
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && rows_live) {
+#pragma unroll
+                    for (int sub = 0; sub < Cfg::DH_N / 32; ++sub) {
+                        const int x = j * Cfg::DH_N + 32 * sub;
+                        if (x < D)
+                            tma_reduce_add_2d(&tmDh, stage0 + (uint32_t)sub * Cfg::EPI_BUF_BYTES, x,
+                                              row0 + 32 * q);
+                    }
+                    bulk_commit_group();
+                }
+                __syncwarp();
             }
         }
-        st.drain();
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();
