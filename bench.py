@@ -418,7 +418,8 @@ def main():
                     "frac_of_burst": ach / peaks["bf16_tflops"],
                     "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
                     "flops_per_launch": fl_launch, "ms_per_launch": dom_ms,
-                    "traffic": traffic_for(dom, args.workload)}
+                    # the committed summaries are of whole-batch launches
+                    "traffic": traffic_for(dom, args.workload) if args.tokens == 0 else None}
         else:
             # fp32 runs on the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flop
             # (FMA) x 1.965 GHz (max SM clock) = 74.4 TFLOP/s
