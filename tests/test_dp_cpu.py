@@ -169,3 +169,54 @@ def test_rank_leaving_between_steps_fails_the_next_step(total):
             dt, outcome = f.read().splitlines()[:2]
     assert outcome != "completed", "the step completed without its peer"
     assert float(dt) < 6 * PG_TIMEOUT_S, f"took {dt} s to fail: {outcome}"
+
+
+# ------------------------------------------------------------ uneven shards, three ranks
+UNEVEN_CUTS = (0, 7, 7 + 21, 40)     # rank 0: 7 tokens, rank 1: 21, rank 2: 12
+
+
+def _uneven_worker(rank, port, outdir, total, world):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from linear_diffusion_cross_b200.dp import fwd_bwd_data_parallel
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        H, W, y, p, b = _case(seed=3)
+        y = y.copy()
+        y[UNEVEN_CUTS[0]:UNEVEN_CUTS[1]] = -100        # rank 0 holds no valid token
+        sl = slice(UNEVEN_CUTS[rank], UNEVEN_CUTS[rank + 1])
+        kw = dict(logit_scale=1.3, label_smoothing=0.05, ignore_index=-100)
+        k = OracleKernels(W.shape[0], kw)
+        out = fwd_bwd_data_parallel(
+            k, torch.from_numpy(H[sl]), torch.from_numpy(W), torch.from_numpy(y[sl]),
+            torch.from_numpy(p[sl]), total=total, grad_out=0.75, bias=torch.from_numpy(b))
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"), loss=out["loss"].numpy(),
+                 dW=out["dW"].numpy(), dH=out["dH"].numpy(), db=out["db"].numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("total", [0.0, 40.0])
+def test_three_uneven_ranks_match_whole_batch(total):
+    """Three ranks with 7, 21 and 12 tokens (the first holding no token that
+    carries a loss): the job-wide count, the summed dW, db and loss and each
+    rank's dH rows equal the oracle on the whole batch."""
+    import oracle.fldce_oracle as O
+    world = len(UNEVEN_CUTS) - 1
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_uneven_worker, args=(_free_port(), d, total, world), nprocs=world,
+                           join=True, start_method="spawn")
+        H, W, y, p, b = _case(seed=3)
+        y = y.copy()
+        y[UNEVEN_CUTS[0]:UNEVEN_CUTS[1]] = -100
+        ref = O.fldce(H, W, y, p, total=total, grad_out=0.75, logit_scale=1.3,
+                      label_smoothing=0.05, bias=b)
+        for rank in range(world):
+            r = np.load(os.path.join(d, f"rank{rank}.npz"))
+            assert abs(float(r["loss"][0]) - ref.loss) <= 1e-12 * abs(ref.loss)
+            assert np.allclose(r["dW"], ref.dW, rtol=1e-11, atol=1e-15)
+            assert np.allclose(r["db"], ref.db, rtol=1e-11, atol=1e-15)
+            sl = slice(UNEVEN_CUTS[rank], UNEVEN_CUTS[rank + 1])
+            assert np.allclose(r["dH"], ref.dH[sl], rtol=1e-11, atol=1e-15)
+        assert np.all(np.load(os.path.join(d, "rank0.npz"))["dH"] == 0.0)

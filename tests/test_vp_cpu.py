@@ -11,11 +11,11 @@ import socket
 import tempfile
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-WORLD = 2
 
 
 class OracleShardKernels:
@@ -73,16 +73,15 @@ def _case():
     return H, W, b, y, p
 
 
-def _worker(rank, port, outdir):
+def _worker(rank, port, outdir, cuts):
     import sys
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     from linear_diffusion_cross_b200.dp import fwd_bwd_vocab_parallel
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
-                            world_size=WORLD)
+                            world_size=len(cuts) - 1)
     try:
         H, W, b, y, p = _case()
-        cut = 17
-        a, e = (0, cut) if rank == 0 else (cut, W.shape[0])
+        a, e = cuts[rank], cuts[rank + 1]
         k = OracleShardKernels(a, W.shape[0], dict(logit_scale=0.9, label_smoothing=0.1))
         out = fwd_bwd_vocab_parallel(k, torch.from_numpy(H), torch.from_numpy(W[a:e]),
                                      torch.from_numpy(y), torch.from_numpy(p), total=0.0,
@@ -93,20 +92,26 @@ def _worker(rank, port, outdir):
         dist.destroy_process_group()
 
 
-def test_vocab_parallel_exchange_matches_whole_vocabulary():
+@pytest.mark.parametrize("cuts", [(0, 17, 41), (0, 5, 30, 41)])
+def test_vocab_parallel_exchange_matches_whole_vocabulary(cuts):
+    """Two shards (17 + 24 rows) and three uneven ones (5 + 25 + 11 rows):
+    every rank's loss and dH equal the oracle's on the whole vocabulary, and
+    its dW and db rows equal the oracle's rows of its shard."""
     import oracle.fldce_oracle as O
+    world = len(cuts) - 1
     with socket.socket() as sk:
         sk.bind(("127.0.0.1", 0))
         port = sk.getsockname()[1]
     with tempfile.TemporaryDirectory() as d:
-        mp.start_processes(_worker, args=(port, d), nprocs=WORLD, join=True,
+        mp.start_processes(_worker, args=(port, d, cuts), nprocs=world, join=True,
                            start_method="spawn")
         H, W, b, y, p = _case()
         ref = O.fldce(H, W, y, p, total=0.0, logit_scale=0.9, label_smoothing=0.1,
                       grad_out=1.3, bias=b)
-        for r in range(WORLD):
+        for r in range(world):
             z = np.load(os.path.join(d, f"r{r}.npz"))
             a, e = int(z["a"]), int(z["e"])
+            assert (a, e) == (cuts[r], cuts[r + 1])
             assert math.isclose(float(z["loss"][0]), ref.loss, rel_tol=1e-12)
             assert np.allclose(z["dH"], ref.dH, rtol=1e-11, atol=1e-15)
             assert np.allclose(z["dW"], ref.dW[a:e], rtol=1e-11, atol=1e-15)
