@@ -101,7 +101,44 @@ def test_full_size(name):
     loss = float(g["loss"][0])
     info["loss"] = abs(loss - loss_ref) / abs(loss_ref)
     assert abs(loss - loss_ref) <= LOSS_RTOL * abs(loss_ref), (loss, loss_ref)
+
+    if name in ("ragged", "large"):
+        # the same batch with the ignored tokens compacted away on the device
+        # (FLDCE_FLAG_SKIP_IGNORED; for large, across its four token chunks)
+        # against the same oracle values
+        del g
+        skip = _run_skip(wl)
+        ls = float(skip["loss"][0])
+        info["skip_loss"] = abs(ls - loss_ref) / abs(loss_ref)
+        assert abs(ls - loss_ref) <= LOSS_RTOL * abs(loss_ref), (ls, loss_ref)
+        e = maxabs_err(f64(skip["dW"])[vr], dWr)
+        info["skip_dW"] = e
+        assert e <= GRAD_TOL["bf16"], f"skip dW err {e}"
+        vrows = rows[valid[rows]]
+        e = maxabs_err(f64(skip["dH"])[vrows], ref.dH[valid[rows]])
+        info["skip_dH"] = e
+        assert e <= GRAD_TOL["bf16"], f"skip dH err {e}"
+        ign = torch.from_numpy(~valid)
+        assert torch.count_nonzero(skip["dH"][ign]) == 0
+        assert torch.isnan(skip["lse"][ign]).all()
+        lt = skip["loss_per_token"].double().numpy()
+        assert maxabs_err(lt, lt_all) <= ROW_TOL["bf16"]
     print(name, info)
+
+
+def _run_skip(wl):
+    from linear_diffusion_cross_b200 import binding as B
+    dev = torch.device("cuda")
+    plan = B.Plan(wl.D, wl.V, wl.N, chunk_N=wl.chunk_n, logit_scale=wl.logit_scale,
+                  label_smoothing=wl.label_smoothing, ignore_index=wl.ignore_index,
+                  skip_ignored=True, device=dev)
+    out = plan.fwd_bwd(wl.H.to(dev), wl.W.to(dev), wl.target.to(dev), wl.p_mask.to(dev),
+                       wl.total, wl.grad_out)
+    torch.cuda.synchronize()
+    res = {k: v.cpu() for k, v in out.items()}
+    assert res["err"].tolist() == [0, 0]
+    plan.close()
+    return res
 
 
 def test_full_size_headline_skip_ignored():
