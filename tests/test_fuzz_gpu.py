@@ -1,9 +1,11 @@
 """Seeded random configurations against the float64 oracle: shapes with
 ragged tiles in every dimension, and random combinations of the options
 (label smoothing, negative and large logit scales, bias, p_mask or none,
-explicit or counted normaliser, chunking, fp32 dW / dH, compacted tokens,
-the fp32 element type).  Each case is small enough for the oracle to take a
-fraction of a second; the list is fixed by its seeds."""
+explicit or counted normaliser, chunking -- including chunk starts off the
+16-byte boundary of the per-token arrays --, fp32 dW / dH, compacted tokens,
+the fused sweep 2 + dH kernel, the fp32 element type).  Each case is small
+enough for the oracle to take a fraction of a second; the list is fixed by
+its seeds."""
 import numpy as np
 import pytest
 import torch
@@ -35,12 +37,18 @@ def _case(seed):
     skip = (not fp32) and bool(rng.integers(0, 3) == 0)
     dw_fp32 = bool(rng.integers(0, 2))
     dh_fp32 = (not fp32) and (not skip) and bool(rng.integers(0, 3) == 0)
-    return fp32, N, D, V, opts, chunk, bias, p_none, skip, dw_fp32, dh_fp32
+    fused = False
+    if seed >= 28:
+        # later seeds: chunk starts off the 16-byte boundary of the per-token
+        # arrays, and the fused sweep 2 + dH kernel among the options
+        chunk = int(rng.choice([0, 33, 99, 130]))
+        fused = (not fp32) and (not skip) and bool(rng.integers(0, 2))
+    return fp32, N, D, V, opts, chunk, bias, p_none, skip, dw_fp32, dh_fp32, fused
 
 
-@pytest.mark.parametrize("seed", range(28))
+@pytest.mark.parametrize("seed", range(48))
 def test_random_configuration(seed):
-    fp32, N, D, V, opts, chunk, bias, p_none, skip, dw_fp32, dh_fp32 = _case(seed)
+    fp32, N, D, V, opts, chunk, bias, p_none, skip, dw_fp32, dh_fp32, fused = _case(seed)
     dtype = torch.float32 if fp32 else torch.bfloat16
     r = synth.Recipe("fuzz", 1, N, D, V, dtype, 0.1, 1e-3)
     wl = synth.make(r, seed, **opts)
@@ -48,7 +56,7 @@ def test_random_configuration(seed):
         if bias else None
     plan = B.Plan(D, V, N, dtype=dtype, chunk_N=chunk, logit_scale=wl.logit_scale,
                   label_smoothing=wl.label_smoothing, dw_fp32=dw_fp32, dh_fp32=dh_fp32,
-                  skip_ignored=skip, device=DEV)
+                  skip_ignored=skip, fused_dh=fused, device=DEV)
     p = None if p_none else wl.p_mask.to(DEV)
     out = plan.fwd_bwd(wl.H.to(DEV), wl.W.to(DEV), wl.target.to(DEV), p, wl.total,
                        wl.grad_out, bias=None if b is None else b.to(DEV), want_argmax=True)
@@ -59,7 +67,7 @@ def test_random_configuration(seed):
                   grad_out=wl.grad_out, bias=None if b is None else f64(b))
     key = "fp32" if fp32 else "bf16"
     ctx = (f"seed {seed}: N={N} D={D} V={V} {opts} chunk={chunk} bias={bias} "
-           f"p_none={p_none} skip={skip} dw_fp32={dw_fp32} dh_fp32={dh_fp32}")
+           f"p_none={p_none} skip={skip} dw_fp32={dw_fp32} dh_fp32={dh_fp32} fused={fused}")
     loss = float(out["loss"][0])
     assert abs(loss - ref.loss) <= LOSS_RTOL * abs(ref.loss) + 1e-6, ctx
     assert maxabs_err(f64(out["dH"]), ref.dH) <= GRAD_TOL[key], ctx
