@@ -89,7 +89,9 @@ extern "C" {
  * dH).  The page runs dx = dlogits @ weight on the gradient it wrote over
  * the logits (fused_linear_cross_entropy_forward's chunk loop); this is the
  * on-chip form of that step.  An alternative design, measured against the
- * default (staged G read back by a separate dH GEMM), not the default. */
+ * default (staged G read back by a separate dH GEMM) and not the default:
+ * its fp32 partials move 2 D / 256 times the bytes the staged dH reads
+ * back, and it ran about twice as long as sweep 2 + dH on B200. */
 #define FLDCE_FLAG_FUSED_DH      0x10u
 
 typedef struct fldce_plan* fldce_handle;
