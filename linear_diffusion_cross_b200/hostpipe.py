@@ -10,7 +10,10 @@ the other slot.  Events order the three streams:
 * a slot's inputs are refilled only after the call that read them finished;
 * a call starts only after its slot's inputs have landed, and only after the
   download of the results that slot held two steps earlier has finished;
-* a download starts only after the call that wrote the results finished.
+* a download starts only after the call that wrote the results finished --
+  except dW's: the library computes the last chunk's dW before its dH and
+  records an event as soon as dW is final, and dW (the largest result)
+  starts downloading then, while dH is still being computed.
 
 Every step still moves all of its inputs and results; the copies overlap the
 neighbouring steps' compute (PCIe upload and download run concurrently on
@@ -50,6 +53,11 @@ class HostPipeline:
         self.filled = [torch.cuda.Event() for _ in range(2)]    # inputs landed
         self.done = [torch.cuda.Event() for _ in range(2)]      # the call finished
         self.fetched = [torch.cuda.Event() for _ in range(2)]   # results downloaded
+        # dW final (recorded by the library by handle, so created up front)
+        self.dw_ready = [torch.cuda.Event() for _ in range(2)]
+        cur = torch.cuda.current_stream(dev)
+        for e in self.dw_ready:
+            e.record(cur)
         self._last = 0
 
     @property
@@ -88,16 +96,24 @@ class HostPipeline:
         stream.wait_event(self.filled[slot])
         stream.wait_event(self.fetched[slot])      # results of two steps ago are out
         self.plan.fwd_bwd(s["H"], s["W"], s["y"], s["p"], total, grad_out, out=s["out"],
-                          stream=stream)
+                          stream=stream, dw_ready_event=self.dw_ready[slot])
         self.done[slot].record(stream)
 
     def _fetch(self, slot: int, copies) -> None:
-        """Copy (key, host tensor) pairs of the slot's results to the host."""
+        """Copy (key, host tensor) pairs of the slot's results to the host:
+        dW as soon as it is final, the rest once the call has finished."""
         fs = self.fetch_stream
-        fs.wait_event(self.done[slot])
         out = self.slots[slot]["out"]
+        early = [(k, t) for k, t in copies if k == "dW"]
+        late = [(k, t) for k, t in copies if k != "dW"]
+        if early:
+            fs.wait_event(self.dw_ready[slot])
+            with torch.cuda.stream(fs):
+                for k, t in early:
+                    t.copy_(out[k], non_blocking=True)
+        fs.wait_event(self.done[slot])
         with torch.cuda.stream(fs):
-            for k, t in copies:
+            for k, t in late:
                 t.copy_(out[k], non_blocking=True)
         self.fetched[slot].record(fs)
 
